@@ -1,0 +1,126 @@
+// Shared device helpers and the workspace layout of liblora_b200.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lora.h"
+
+namespace lora {
+
+constexpr int kItemTokens = 16;     // tokens per work item of the per-token kernels
+constexpr int kMaxRank = 64;
+
+// ---------------------------------------------------------------------------
+// Workspace ("meta") layout.  Offsets are multiples of 256 bytes.
+//   [0, 256)       header
+//   slot_off       int32 [S + 2]: slot g's tokens are perm[slot_off[g] ..
+//                  slot_off[g+1]); [slot_off[S], slot_off[S+1]) = the tokens
+//                  without an adapter
+//   perm           int32 [T]
+//   items          int4 [max_items]: {slot (-1 = none), begin, end, flags}
+// ---------------------------------------------------------------------------
+struct MetaHeader {
+  int bad_index;      // count of indices outside [-1, S) (accumulates)
+  int bad_meta;       // malformed segment lists, or metadata built for other
+                      // sizes than the call's (accumulates)
+  int n_items;        // items in the work list
+  int n_active;       // tokens with an adapter
+  int T, S;           // sizes the metadata was built for
+  int pad[58];
+};
+static_assert(sizeof(MetaHeader) == 256, "header is 256 bytes");
+
+enum ItemFlags { kItemDirect = 1 };   // token = position (segments), no perm
+
+struct MetaLayout {
+  size_t off_slot, off_perm, off_items, total;
+  int max_items;
+  __host__ __device__ static size_t a256(size_t v) { return (v + 255) & ~size_t(255); }
+  __host__ __device__ MetaLayout(int T, int S) {
+    int tt = T > 0 ? T : 1;
+    off_slot = 256;
+    off_perm = off_slot + a256(sizeof(int) * (size_t)(S + 2));
+    off_items = off_perm + a256(sizeof(int) * (size_t)tt);
+    // per-token grouping: <= T/16 + (S + 1) items; segments: <= T/16 + n_seg
+    // with n_seg <= T + 1.
+    max_items = T / kItemTokens + (S + 1 > T + 1 ? S + 1 : T + 1) + 2;
+    total = off_items + a256(sizeof(int4) * (size_t)max_items);
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Element types
+// ---------------------------------------------------------------------------
+template <typename E> struct Elem;
+template <> struct Elem<__half> {
+  // 8 packed halves (16 bytes) -> 8 floats
+  static __device__ __forceinline__ void to_f32(const uint4& v, float* f) {
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float2 p = __half22float2(h[k]);
+      f[2 * k] = p.x;
+      f[2 * k + 1] = p.y;
+    }
+  }
+  static __device__ __forceinline__ float to_f32(uint16_t b) {
+    return __half2float(__ushort_as_half(b));
+  }
+  static __device__ __forceinline__ uint16_t from_f32(float f) {
+    return __half_as_ushort(__float2half_rn(f));
+  }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ void to_f32(const uint4& v, float* f) {
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      f[2 * k] = __uint_as_float(w[k] << 16);
+      f[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+  }
+  static __device__ __forceinline__ float to_f32(uint16_t b) {
+    return __uint_as_float(((uint32_t)b) << 16);
+  }
+  static __device__ __forceinline__ uint16_t from_f32(float f) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+  }
+};
+
+// 16-byte read-only global load (no L1 allocation for streaming data).
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint4 ldg_nc(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Work items of the metadata, or 0 (and the error counted) when the metadata
+// was built for other sizes than the call's: item token positions are then not
+// known to lie inside this call's buffers.
+__device__ __forceinline__ int checked_items(const char* meta, int T, int S) {
+  const MetaHeader* h = reinterpret_cast<const MetaHeader*>(meta);
+  if (h->T == T && h->S == S) return h->n_items;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+    atomicAdd(const_cast<int*>(&h->bad_meta), 1);
+  return 0;
+}
+
+}  // namespace lora

@@ -1,0 +1,58 @@
+// Host-side launchers shared between the C ABI (lora_api.cu) and the kernel
+// files.  Not part of the public interface.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lora.h"
+
+namespace lora {
+
+struct ShrinkArgs {
+  const void* x;
+  int64_t ldx;
+  const void* A[LORA_MAX_SLICES];
+  float* buf;
+  int T, D, r, S, n_slices;
+  const char* meta;
+};
+
+struct ExpandArgs {
+  const float* buf;
+  int64_t buf_slice_stride;
+  const void* B[LORA_MAX_SLICES];
+  int D_out[LORA_MAX_SLICES];
+  int64_t y_col_off[LORA_MAX_SLICES];
+  int chunk_base[LORA_MAX_SLICES + 1];   // prefix of column chunks per slice
+  float scale;
+  void* y;
+  int64_t ldy;
+  int T, r, S, n_slices;
+  const char* meta;
+};
+
+struct SegArgs {
+  const int32_t* seg_starts;
+  const int32_t* seg_adapter;
+  int n_seg;
+};
+
+size_t group_smem_bytes(int S);
+cudaError_t launch_group(int T, int S, const int32_t* idx, void* meta, cudaStream_t st);
+cudaError_t launch_segment_items(int T, int S, int n_seg, const int32_t* seg_starts,
+                                 const int32_t* seg_adapter, void* meta, cudaStream_t st);
+
+// CUDA-core kernels over the work list in meta (per-token or segment items).
+cudaError_t launch_shrink_items(lora_dtype dt, const ShrinkArgs& a, int max_items,
+                                cudaStream_t st);
+cudaError_t launch_expand_items(lora_dtype dt, ExpandArgs a, int max_items, cudaStream_t st);
+
+// tcgen05 tensor-core kernels for segments.  Return cudaErrorNotSupported if
+// the shape has no tensor-core path (the caller then uses the item kernels).
+cudaError_t launch_shrink_segment_tc(lora_dtype dt, const ShrinkArgs& a, const SegArgs& s,
+                                     cudaStream_t st);
+cudaError_t launch_expand_segment_tc(lora_dtype dt, const ExpandArgs& a, const SegArgs& s,
+                                     cudaStream_t st);
+
+}  // namespace lora

@@ -1,0 +1,251 @@
+// extern "C" entry points of liblora_b200.so: host-side argument checks and
+// dispatch to the kernels.  See include/lora.h for the contract of each call.
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+using namespace lora;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool rank_ok(int r) { return r == 8 || r == 16 || r == 32 || r == 64; }
+
+lora_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA; }
+
+lora_status check_common(lora_dtype dt, int T, int r, int S, int n_slices, const void* meta,
+                         size_t meta_bytes) {
+  if (dt != LORA_F16 && dt != LORA_BF16) return LORA_ERR_INVALID_ARG;
+  if (T < 0 || S < 0 || n_slices < 0) return LORA_ERR_INVALID_ARG;
+  if (T > LORA_MAX_TOKENS || S < 1 || S > LORA_MAX_SLOTS) return LORA_ERR_UNSUPPORTED;
+  if (n_slices < 1 || n_slices > LORA_MAX_SLICES || !rank_ok(r)) return LORA_ERR_UNSUPPORTED;
+  if (meta == nullptr) return LORA_ERR_INVALID_ARG;
+  if (!aligned16(meta)) return LORA_ERR_MISALIGNED;
+  if (meta_bytes < lora_workspace_bytes(T, S)) return LORA_ERR_INVALID_ARG;
+  return LORA_OK;
+}
+
+lora_status check_shrink(lora_dtype dt, int T, int D, int r, int S, int n_slices,
+                         const void* x, int64_t ldx, const void* const* A, const float* buf,
+                         const void* meta, size_t meta_bytes) {
+  lora_status s = check_common(dt, T, r, S, n_slices, meta, meta_bytes);
+  if (s != LORA_OK) return s;
+  if (D <= 0) return LORA_ERR_INVALID_ARG;
+  if (T == 0) return LORA_OK;   // nothing to read or write
+  if (A == nullptr || x == nullptr || buf == nullptr) return LORA_ERR_INVALID_ARG;
+  if (D % 8 != 0) return LORA_ERR_MISALIGNED;
+  if (ldx < D) return LORA_ERR_INVALID_ARG;
+  if (ldx % 8 != 0 || !aligned16(x) || !aligned16(buf)) return LORA_ERR_MISALIGNED;
+  for (int i = 0; i < n_slices; ++i) {
+    if (A[i] == nullptr) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(A[i])) return LORA_ERR_MISALIGNED;
+  }
+  return LORA_OK;
+}
+
+lora_status check_expand(lora_dtype dt, int T, int r, int S, int n_slices, const float* buf,
+                         int64_t buf_slice_stride, const void* const* B, const int32_t* D_out,
+                         const void* y, int64_t ldy, const int64_t* y_col_off,
+                         const void* meta, size_t meta_bytes) {
+  lora_status s = check_common(dt, T, r, S, n_slices, meta, meta_bytes);
+  if (s != LORA_OK) return s;
+  if (T == 0) return LORA_OK;   // nothing to read or write
+  if (buf == nullptr || B == nullptr || D_out == nullptr || y == nullptr || y_col_off == nullptr)
+    return LORA_ERR_INVALID_ARG;
+  if (buf_slice_stride < 0) return LORA_ERR_INVALID_ARG;
+  if (buf_slice_stride > 0 && buf_slice_stride < (int64_t)T * r) return LORA_ERR_INVALID_ARG;
+  if (buf_slice_stride % 4 != 0 || !aligned16(buf) || !aligned16(y) || ldy % 8 != 0)
+    return LORA_ERR_MISALIGNED;
+  for (int i = 0; i < n_slices; ++i) {
+    if (B[i] == nullptr || D_out[i] <= 0 || y_col_off[i] < 0) return LORA_ERR_INVALID_ARG;
+    if (D_out[i] % 8 != 0 || y_col_off[i] % 8 != 0 || !aligned16(B[i]))
+      return LORA_ERR_MISALIGNED;
+    if (y_col_off[i] + D_out[i] > ldy) return LORA_ERR_INVALID_ARG;
+    for (int k = 0; k < i; ++k) {   // output slices must not overlap
+      int64_t a0 = y_col_off[i], a1 = a0 + D_out[i];
+      int64_t b0 = y_col_off[k], b1 = b0 + D_out[k];
+      if (a0 < b1 && b0 < a1) return LORA_ERR_INVALID_ARG;
+    }
+  }
+  return LORA_OK;
+}
+
+lora_status check_segments(int T, int n_seg, const int32_t* seg_starts,
+                           const int32_t* seg_adapter) {
+  if (n_seg < 0 || n_seg > T + 1) return LORA_ERR_INVALID_ARG;
+  if (T == 0) return LORA_OK;
+  if (seg_starts == nullptr || seg_adapter == nullptr) return LORA_ERR_INVALID_ARG;
+  if (n_seg == 0 && T != 0) return LORA_ERR_INVALID_ARG;
+  return LORA_OK;
+}
+
+int max_items_tokens(int T, int S) { return T / kItemTokens + S + 2; }
+int max_items_segments(int T, int n_seg) { return T / kItemTokens + n_seg + 2; }
+
+}  // namespace
+
+extern "C" {
+
+size_t lora_workspace_bytes(int T, int S) {
+  if (T < 0 || T > LORA_MAX_TOKENS || S < 1 || S > LORA_MAX_SLOTS) return 0;
+  return MetaLayout(T, S).total;
+}
+
+lora_status lora_workspace_reset(void* meta, size_t meta_bytes, lora_stream_t stream) {
+  if (meta == nullptr) return LORA_ERR_INVALID_ARG;
+  return from_cuda(cudaMemsetAsync(meta, 0, meta_bytes, (cudaStream_t)stream));
+}
+
+lora_status lora_group(int T, int S, const int32_t* idx, void* meta, size_t meta_bytes,
+                       lora_stream_t stream) {
+  if (T < 0 || S < 0) return LORA_ERR_INVALID_ARG;
+  if (T > LORA_MAX_TOKENS || S < 1 || S > LORA_MAX_SLOTS) return LORA_ERR_UNSUPPORTED;
+  if (meta == nullptr || (T > 0 && idx == nullptr)) return LORA_ERR_INVALID_ARG;
+  if (!aligned16(meta)) return LORA_ERR_MISALIGNED;
+  if (meta_bytes < lora_workspace_bytes(T, S)) return LORA_ERR_INVALID_ARG;
+  cudaGetLastError();
+  return from_cuda(launch_group(T, S, idx, meta, (cudaStream_t)stream));
+}
+
+lora_status lora_shrink(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
+                        const void* x, int64_t ldx, const void* const* A, float* buf,
+                        int has_active, const void* meta, size_t meta_bytes,
+                        lora_stream_t stream) {
+  lora_status s = check_shrink(dtype, T, D, r, S, n_slices, x, ldx, A, buf, meta, meta_bytes);
+  if (s != LORA_OK) return s;
+  if (!has_active || T == 0) return LORA_OK;
+  ShrinkArgs a = {};
+  a.x = x;
+  a.ldx = ldx;
+  for (int i = 0; i < n_slices; ++i) a.A[i] = A[i];
+  a.buf = buf;
+  a.T = T; a.D = D; a.r = r; a.S = S; a.n_slices = n_slices;
+  a.meta = static_cast<const char*>(meta);
+  cudaGetLastError();
+  return from_cuda(launch_shrink_items(dtype, a, max_items_tokens(T, S), (cudaStream_t)stream));
+}
+
+static void fill_expand(ExpandArgs& a, int T, int r, int S, int n_slices, const float* buf,
+                        int64_t buf_slice_stride, const void* const* B, const int32_t* D_out,
+                        float scale, void* y, int64_t ldy, const int64_t* y_col_off,
+                        const void* meta) {
+  a.buf = buf;
+  a.buf_slice_stride = buf_slice_stride;
+  for (int i = 0; i < n_slices; ++i) {
+    a.B[i] = B[i];
+    a.D_out[i] = D_out[i];
+    a.y_col_off[i] = y_col_off[i];
+  }
+  a.scale = scale;
+  a.y = y;
+  a.ldy = ldy;
+  a.T = T; a.r = r; a.S = S; a.n_slices = n_slices;
+  a.meta = static_cast<const char*>(meta);
+}
+
+lora_status lora_expand(lora_dtype dtype, int T, int r, int S, int n_slices,
+                        const float* buf, int64_t buf_slice_stride, const void* const* B,
+                        const int32_t* D_out, float scale, void* y, int64_t ldy,
+                        const int64_t* y_col_off, int has_active, const void* meta,
+                        size_t meta_bytes, lora_stream_t stream) {
+  lora_status s = check_expand(dtype, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, y,
+                               ldy, y_col_off, meta, meta_bytes);
+  if (s != LORA_OK) return s;
+  if (!has_active || T == 0) return LORA_OK;
+  ExpandArgs a = {};
+  fill_expand(a, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, scale, y, ldy, y_col_off,
+              meta);
+  cudaGetLastError();
+  return from_cuda(launch_expand_items(dtype, a, max_items_tokens(T, S), (cudaStream_t)stream));
+}
+
+lora_status lora_shrink_segment(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
+                                const void* x, int64_t ldx, const void* const* A,
+                                const int32_t* seg_starts, const int32_t* seg_adapter,
+                                int n_seg, float* buf, int has_active, void* meta,
+                                size_t meta_bytes, lora_stream_t stream) {
+  lora_status s = check_shrink(dtype, T, D, r, S, n_slices, x, ldx, A, buf, meta, meta_bytes);
+  if (s != LORA_OK) return s;
+  s = check_segments(T, n_seg, seg_starts, seg_adapter);
+  if (s != LORA_OK) return s;
+  if (!has_active || T == 0) return LORA_OK;
+  ShrinkArgs a = {};
+  a.x = x;
+  a.ldx = ldx;
+  for (int i = 0; i < n_slices; ++i) a.A[i] = A[i];
+  a.buf = buf;
+  a.T = T; a.D = D; a.r = r; a.S = S; a.n_slices = n_slices;
+  a.meta = static_cast<const char*>(meta);
+  SegArgs sg = {seg_starts, seg_adapter, n_seg};
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaGetLastError();
+  cudaError_t e = launch_shrink_segment_tc(dtype, a, sg, st);
+  if (e == cudaErrorNotSupported) {
+    cudaGetLastError();
+    e = launch_segment_items(T, S, n_seg, seg_starts, seg_adapter, meta, st);
+    if (e == cudaSuccess) e = launch_shrink_items(dtype, a, max_items_segments(T, n_seg), st);
+  }
+  return from_cuda(e);
+}
+
+lora_status lora_expand_segment(lora_dtype dtype, int T, int r, int S, int n_slices,
+                                const float* buf, int64_t buf_slice_stride,
+                                const void* const* B, const int32_t* D_out,
+                                const int32_t* seg_starts, const int32_t* seg_adapter,
+                                int n_seg, float scale, void* y, int64_t ldy,
+                                const int64_t* y_col_off, int has_active, void* meta,
+                                size_t meta_bytes, lora_stream_t stream) {
+  lora_status s = check_expand(dtype, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, y,
+                               ldy, y_col_off, meta, meta_bytes);
+  if (s != LORA_OK) return s;
+  s = check_segments(T, n_seg, seg_starts, seg_adapter);
+  if (s != LORA_OK) return s;
+  if (!has_active || T == 0) return LORA_OK;
+  ExpandArgs a = {};
+  fill_expand(a, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, scale, y, ldy, y_col_off,
+              meta);
+  SegArgs sg = {seg_starts, seg_adapter, n_seg};
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaGetLastError();
+  cudaError_t e = launch_expand_segment_tc(dtype, a, sg, st);
+  if (e == cudaErrorNotSupported) {
+    cudaGetLastError();
+    e = launch_segment_items(T, S, n_seg, seg_starts, seg_adapter, meta, st);
+    if (e == cudaSuccess) e = launch_expand_items(dtype, a, max_items_segments(T, n_seg), st);
+  }
+  return from_cuda(e);
+}
+
+lora_status lora_check_errors(void* meta, size_t meta_bytes, lora_stream_t stream) {
+  if (meta == nullptr || meta_bytes < sizeof(MetaHeader)) return LORA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LORA_ERR_CUDA;
+  int h[2] = {0, 0};
+  if (cudaMemcpy(h, meta, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return LORA_ERR_CUDA;
+  if (h[0] || h[1]) {
+    int z[2] = {0, 0};
+    if (cudaMemcpy(meta, z, sizeof(z), cudaMemcpyHostToDevice) != cudaSuccess)
+      return LORA_ERR_CUDA;
+    return LORA_ERR_BAD_INDEX;
+  }
+  return LORA_OK;
+}
+
+const char* lora_status_string(lora_status status) {
+  switch (status) {
+    case LORA_OK: return "LORA_OK";
+    case LORA_ERR_INVALID_ARG: return "LORA_ERR_INVALID_ARG";
+    case LORA_ERR_UNSUPPORTED: return "LORA_ERR_UNSUPPORTED";
+    case LORA_ERR_MISALIGNED: return "LORA_ERR_MISALIGNED";
+    case LORA_ERR_CUDA: return "LORA_ERR_CUDA";
+    case LORA_ERR_BAD_INDEX: return "LORA_ERR_BAD_INDEX";
+  }
+  return "LORA_ERR_UNKNOWN";
+}
+
+const char* lora_build_info(void) { return "liblora_b200 sm_100a 0.1"; }
+
+}  // extern "C"

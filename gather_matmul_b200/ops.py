@@ -1,0 +1,156 @@
+"""Python binding of the multi-LoRA shrink / expand C ABI.
+
+Argument marshalling only: each function reads shapes, strides and device
+pointers off torch tensors, passes them to liblora_b200.so on the current
+torch CUDA stream, and raises LoraError on a non-OK status.  Every step of the
+computation runs in the library's CUDA kernels; torch supplies device memory
+and streams.
+
+  group(idx, S, meta)                          per-batch group-by-slot metadata
+  shrink(x, A, buf, meta)                      buf[i] = per-token x . A_i[idx]^T
+  expand(buf, B, y, meta, scale)               y[:, slice_i] += scale buf_i . B_i[idx]^T
+  shrink_segment / expand_segment              the same with segments
+  check_errors(meta)                           device-side bad-index report
+"""
+import ctypes
+from typing import Optional, Sequence
+
+import torch
+
+from . import _lib
+
+_DT = {torch.float16: _lib.LORA_F16, torch.bfloat16: _lib.LORA_BF16}
+
+
+class LoraError(RuntimeError):
+    def __init__(self, call, status):
+        self.status = status
+        super().__init__(f"{call} failed: {_lib.status_string(status)} ({status})")
+
+
+def _check(call, status):
+    if status != _lib.LORA_OK:
+        raise LoraError(call, status)
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+
+
+def _ptrs(ts):
+    return (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+
+
+def _dtype(t):
+    if t.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {t.dtype}; fp16 or bf16")
+    return _DT[t.dtype]
+
+
+def workspace_bytes(T: int, S: int) -> int:
+    return _lib.load().lora_workspace_bytes(int(T), int(S))
+
+
+def workspace(T: int, S: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace ("meta") for batches of up to T tokens over S slots."""
+    n = workspace_bytes(T, S)
+    if n == 0:
+        raise LoraError("lora_workspace_bytes", _lib.LORA_ERR_UNSUPPORTED)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def group(idx: torch.Tensor, S: int, meta: torch.Tensor, stream=None):
+    """Group-by-slot metadata of one batch's int32 adapter indices (-1 = none)."""
+    if idx.dtype != torch.int32 or not idx.is_contiguous():
+        raise TypeError("idx must be a contiguous int32 tensor")
+    _check("lora_group", _lib.load().lora_group(idx.numel(), int(S), _ptr(idx), _ptr(meta),
+                                                meta.numel(), _stream(stream)))
+
+
+def _xinfo(x):
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be [T, D] with unit column stride")
+    return x.shape[0], x.shape[1], x.stride(0)
+
+
+def shrink(x: torch.Tensor, A: Sequence[torch.Tensor], buf: torch.Tensor, meta: torch.Tensor,
+           has_active: bool = True, stream=None) -> torch.Tensor:
+    """buf[i, t, :] = x[t] . A[i][idx[t]]^T (0 for tokens without an adapter).
+
+    A: list of [S, r, D] stacks; buf: float32 [len(A), T, r]; meta from group()."""
+    T, D, ldx = _xinfo(x)
+    S, r, _ = A[0].shape
+    _check("lora_shrink", _lib.load().lora_shrink(
+        _dtype(x), T, D, r, S, len(A), _ptr(x), ldx, _ptrs(A), _ptr(buf), int(bool(has_active)),
+        _ptr(meta), meta.numel(), _stream(stream)))
+    return buf
+
+
+def _expand_common(buf, B, y, y_col_off, buf_slice_stride):
+    if y.dim() != 2 or y.stride(1) != 1:
+        raise ValueError("y must be [T, ldy] with unit column stride")
+    T, ldy = y.shape[0], y.stride(0)
+    S, _, r = B[0].shape
+    n = len(B)
+    d_out = (ctypes.c_int32 * n)(*[b.shape[1] for b in B])
+    if y_col_off is None:
+        offs, c = [], 0
+        for b in B:
+            offs.append(c)
+            c += b.shape[1]
+        y_col_off = offs
+    off = (ctypes.c_int64 * n)(*[int(v) for v in y_col_off])
+    if buf_slice_stride is None:
+        buf_slice_stride = 0 if buf.dim() == 2 else buf.stride(0)
+    return T, ldy, S, r, n, d_out, off, int(buf_slice_stride)
+
+
+def expand(buf: torch.Tensor, B: Sequence[torch.Tensor], y: torch.Tensor, meta: torch.Tensor,
+           scale: float = 1.0, y_col_off=None, buf_slice_stride=None, has_active: bool = True,
+           stream=None) -> torch.Tensor:
+    """y[t, off_i:off_i+D_out_i] += scale * buf[i, t] . B[i][idx[t]]^T, in place.
+
+    B: list of [S, D_out_i, r]; buf: float32 [n, T, r] (or [T, r] shared by
+    every slice); y: [T, >= sum D_out] fp16/bf16."""
+    T, ldy, S, r, n, d_out, off, stride = _expand_common(buf, B, y, y_col_off, buf_slice_stride)
+    _check("lora_expand", _lib.load().lora_expand(
+        _dtype(y), T, r, S, n, _ptr(buf), stride, _ptrs(B), d_out, ctypes.c_float(scale),
+        _ptr(y), ldy, off, int(bool(has_active)), _ptr(meta), meta.numel(), _stream(stream)))
+    return y
+
+
+def shrink_segment(x, A, seg_starts, seg_adapter, buf, meta, has_active=True, stream=None):
+    """shrink() with adapters given by segments (int32 CSR starts [n+1], adapters [n])."""
+    T, D, ldx = _xinfo(x)
+    S, r, _ = A[0].shape
+    _check("lora_shrink_segment", _lib.load().lora_shrink_segment(
+        _dtype(x), T, D, r, S, len(A), _ptr(x), ldx, _ptrs(A), _ptr(seg_starts),
+        _ptr(seg_adapter), seg_adapter.numel(), _ptr(buf), int(bool(has_active)), _ptr(meta),
+        meta.numel(), _stream(stream)))
+    return buf
+
+
+def expand_segment(buf, B, seg_starts, seg_adapter, y, meta, scale=1.0, y_col_off=None,
+                   buf_slice_stride=None, has_active=True, stream=None):
+    """expand() with adapters given by segments."""
+    T, ldy, S, r, n, d_out, off, stride = _expand_common(buf, B, y, y_col_off, buf_slice_stride)
+    _check("lora_expand_segment", _lib.load().lora_expand_segment(
+        _dtype(y), T, r, S, n, _ptr(buf), stride, _ptrs(B), d_out, _ptr(seg_starts),
+        _ptr(seg_adapter), seg_adapter.numel(), ctypes.c_float(scale), _ptr(y), ldy, off,
+        int(bool(has_active)), _ptr(meta), meta.numel(), _stream(stream)))
+    return y
+
+
+def check_errors(meta: torch.Tensor, stream=None) -> int:
+    """Synchronise and return the library status for device-detected bad
+    indices / segments since the last check (0 = LORA_OK); clears them."""
+    return _lib.load().lora_check_errors(_ptr(meta), meta.numel(), _stream(stream))
+
+
+def build_info() -> str:
+    return _lib.load().lora_build_info().decode()

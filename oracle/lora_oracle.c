@@ -96,13 +96,31 @@ static double dec_bf16(uint16_t b) {
   return sign ? -v : v;
 }
 
+/* Every 16-bit pattern decoded once with the definitions above, then looked
+ * up (the values are the same; the table only avoids re-deriving them for
+ * each of the billions of products at full size). */
+static double table_f16[65536], table_bf16[65536];
+static int tables_ready = 0;
+
+static void init_tables(void) {
+  if (tables_ready) return;
+  for (int b = 0; b < 65536; ++b) {
+    table_f16[b] = dec_f16((uint16_t)b);
+    table_bf16[b] = dec_bf16((uint16_t)b);
+  }
+  tables_ready = 1;
+}
+
 static double dec(int dtype, uint16_t bits) {
+  return dtype == LO_BF16 ? table_bf16[bits] : table_f16[bits];
+}
+
+double lo_decode(int dtype, uint16_t bits) {
   return dtype == LO_BF16 ? dec_bf16(bits) : dec_f16(bits);
 }
 
-double lo_decode(int dtype, uint16_t bits) { return dec(dtype, bits); }
-
 void lo_decode_array(int dtype, const uint16_t* in, double* out, int64_t n) {
+  init_tables();
   for (int64_t k = 0; k < n; ++k) out[k] = dec(dtype, in[k]);
 }
 
@@ -156,6 +174,7 @@ int lo_group_by_slot(int T, int S, const int32_t* idx, int32_t* perm,
 int lo_shrink(int dtype, int T, int D, int r, int S, int n_slices,
               const uint16_t* x, int64_t ldx, const uint16_t* const* A,
               const int32_t* idx, double* buf, double* cabs) {
+  init_tables();
   for (int i = 0; i < n_slices; ++i) {
     const uint16_t* Ai = A[i];
 #pragma omp parallel for num_threads(lo_threads) schedule(dynamic, 1)
@@ -197,6 +216,7 @@ int lo_expand(int dtype, int T, int r, int S, int n_slices, const double* buf,
               const int32_t* D_out, const int32_t* idx, double scale,
               const uint16_t* y_old, int64_t ldy, const int64_t* y_col_off,
               double* y_out) {
+  init_tables();
 #pragma omp parallel for num_threads(lo_threads) schedule(dynamic, 1)
   for (int t = 0; t < T; ++t) {
     for (int64_t c = 0; c < ldy; ++c)
