@@ -73,9 +73,9 @@ def group(idx: torch.Tensor, S: int, meta: torch.Tensor, stream=None):
 
 
 def _xinfo(x):
-    if x.dim() != 2 or x.stride(1) != 1:
+    if x.dim() != 2 or (x.numel() > 0 and x.stride(1) != 1):
         raise ValueError("x must be [T, D] with unit column stride")
-    return x.shape[0], x.shape[1], x.stride(0)
+    return x.shape[0], x.shape[1], (x.stride(0) if x.numel() > 0 else x.shape[1])
 
 
 def shrink(x: torch.Tensor, A: Sequence[torch.Tensor], buf: torch.Tensor, meta: torch.Tensor,
@@ -92,9 +92,9 @@ def shrink(x: torch.Tensor, A: Sequence[torch.Tensor], buf: torch.Tensor, meta: 
 
 
 def _expand_common(buf, B, y, y_col_off, buf_slice_stride):
-    if y.dim() != 2 or y.stride(1) != 1:
+    if y.dim() != 2 or (y.numel() > 0 and y.stride(1) != 1):
         raise ValueError("y must be [T, ldy] with unit column stride")
-    T, ldy = y.shape[0], y.stride(0)
+    T, ldy = y.shape[0], (y.stride(0) if y.numel() > 0 else y.shape[1])
     S, _, r = B[0].shape
     n = len(B)
     d_out = (ctypes.c_int32 * n)(*[b.shape[1] for b in B])
