@@ -20,6 +20,7 @@ LORA_BF16 = 1
 LORA_MAX_SLICES = 8
 LORA_MAX_SLOTS = 1024
 LORA_MAX_TOKENS = 1 << 22
+LORA_NOALLOC_MAX_TOKENS = 8192
 
 # Every symbol the header declares, with (restype, argtypes).
 _i32, _i64, _sz, _f32, _vp = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float, ctypes.c_void_p
@@ -36,6 +37,8 @@ SIGNATURES = {
     "lora_expand_segment": (_i32, [_i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _vp,
                                    _i32, _f32, _vp, _i64, _vp, _i32, _vp, _sz, _vp]),
     "lora_check_errors": (_i32, [_vp, _sz, _vp]),
+    "lora_shrink_noalloc": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp,
+                                   _vp, _i32, _vp]),
     "lora_status_string": (ctypes.c_char_p, [_i32]),
     "lora_build_info": (ctypes.c_char_p, []),
 }

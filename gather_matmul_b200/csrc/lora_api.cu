@@ -3,6 +3,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -249,3 +251,78 @@ const char* lora_status_string(lora_status status) {
 const char* lora_build_info(void) { return "liblora_b200 sm_100a 0.1"; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free per-token shrink.
+//
+// For callers that cannot allocate device memory themselves: code running
+// where cudaMalloc is unavailable or forbidden (inside a CUDA-graph capture
+// that must not allocate, an allocator hook, a plugin host that hands out
+// only input and output buffers) and so cannot provide the workspace that
+// lora_group / lora_shrink need.  This entry point keeps that workspace in a
+// fixed device array instead.
+// ---------------------------------------------------------------------------
+namespace {
+
+// Sized for LORA_NOALLOC_MAX_TOKENS tokens over LORA_MAX_SLOTS slots; every
+// GPU that loads the library holds it until the process exits.
+constexpr size_t kNoallocScratchBytes = 176896;
+static_assert(kNoallocScratchBytes == LORA_NOALLOC_SCRATCH_BYTES, "header and library agree");
+static __device__ __align__(256) char g_noalloc_scratch[kNoallocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+
+// Device address of the scratch array for the current device.  The array's
+// name in host code is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+cudaError_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev].store(p, std::memory_order_release);
+  }
+  *out = p;
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" LORA_API lora_status lora_shrink_noalloc(lora_dtype dtype, int T, int D, int r, int S,
+                                                    int n_slices, const void* x, int64_t ldx,
+                                                    const void* const* A, const int32_t* idx,
+                                                    float* buf, int has_active,
+                                                    lora_stream_t stream) {
+  if (T > LORA_NOALLOC_MAX_TOKENS) return LORA_ERR_UNSUPPORTED;
+  if (T >= 0 && S >= 1 && S <= LORA_MAX_SLOTS &&
+      MetaLayout(T, S).total > kNoallocScratchBytes)
+    return LORA_ERR_UNSUPPORTED;
+  // validate against a stand-in workspace size first: nothing is touched yet
+  static const char kFakeMeta[16] __attribute__((aligned(16))) = {0};
+  lora_status s = check_shrink(dtype, T, D, r, S, n_slices, x, ldx, A, buf, kFakeMeta,
+                               kNoallocScratchBytes);
+  if (s != LORA_OK) return s;
+  if (!has_active || T == 0) return LORA_OK;
+  if (idx == nullptr) return LORA_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  cudaGetLastError();
+  if (noalloc_scratch(&scratch) != cudaSuccess) return LORA_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  // the header (error counters, item count) must start at zero each call
+  cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(MetaHeader), st);
+  if (e == cudaSuccess) e = launch_group(T, S, idx, scratch, st);
+  if (e != cudaSuccess) return LORA_ERR_CUDA;
+  ShrinkArgs a = {};
+  a.x = x;
+  a.ldx = ldx;
+  for (int i = 0; i < n_slices; ++i) a.A[i] = A[i];
+  a.buf = buf;
+  a.T = T; a.D = D; a.r = r; a.S = S; a.n_slices = n_slices;
+  a.meta = static_cast<const char*>(scratch);
+  return from_cuda(launch_shrink_items(dtype, a, max_items_tokens(T, S), st));
+}

@@ -146,6 +146,21 @@ def expand_segment(buf, B, seg_starts, seg_adapter, y, meta, scale=1.0, y_col_of
     return y
 
 
+def shrink_noalloc(x: torch.Tensor, A: Sequence[torch.Tensor], idx: torch.Tensor,
+                   buf: torch.Tensor, has_active: bool = True, stream=None) -> torch.Tensor:
+    """group() + shrink() in one call that needs no workspace: the library keeps
+    the grouping scratch in a fixed device array.  For callers that cannot
+    allocate; calls that overlap on the GPU race on that array."""
+    T, D, ldx = _xinfo(x)
+    S, r, _ = A[0].shape
+    if idx.dtype != torch.int32 or not idx.is_contiguous():
+        raise TypeError("idx must be a contiguous int32 tensor")
+    _check("lora_shrink_noalloc", _lib.load().lora_shrink_noalloc(
+        _dtype(x), T, D, r, S, len(A), _ptr(x), ldx, _ptrs(A), _ptr(idx), _ptr(buf),
+        int(bool(has_active)), _stream(stream)))
+    return buf
+
+
 def check_errors(meta: torch.Tensor, stream=None) -> int:
     """Synchronise and return the library status for device-detected bad
     indices / segments since the last check (0 = LORA_OK); clears them."""

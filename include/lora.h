@@ -199,6 +199,37 @@ LORA_API lora_status lora_expand_segment(lora_dtype dtype, int T, int r, int S, 
  */
 LORA_API lora_status lora_check_errors(void* meta, size_t meta_bytes, lora_stream_t stream);
 
+/*
+ * Allocation-free per-token shrink: lora_group + lora_shrink in one call, with
+ * the grouping workspace kept in a fixed array inside the library instead of
+ * caller memory.  The paper has no counterpart; it exists for callers that
+ * cannot allocate device memory (code that runs where cudaMalloc is not
+ * available or not allowed, such as a host that only hands out the input and
+ * output buffers) and so cannot supply `meta`.
+ *
+ *   Arguments as for lora_shrink, plus idx (device int32 [T]) as for
+ *   lora_group; no meta.  Same result as lora_group + lora_shrink.
+ *   Limits: T <= LORA_NOALLOC_MAX_TOKENS and S <= LORA_MAX_SLOTS, else
+ *   LORA_ERR_UNSUPPORTED before anything is enqueued.
+ *   The array is LORA_NOALLOC_SCRATCH_BYTES of device memory that every GPU
+ *   which loads the library holds until the process exits.  The first call on
+ *   a device looks up the array's device address (once per device); make that
+ *   first call before any stream capture.  No cudaMalloc / cudaFree or other
+ *   allocating routine is called.
+ *   Every call shares the one array and it keeps the last call's contents:
+ *   each call clears its header and rebuilds the rest, so calls that overlap
+ *   on the GPU (different streams, or different host threads on one device)
+ *   race and give wrong results; order them.  Indices outside [-1, S) are
+ *   treated as -1 and are not reported (there is no caller workspace to hold
+ *   the error counter).
+ */
+#define LORA_NOALLOC_MAX_TOKENS 8192
+#define LORA_NOALLOC_SCRATCH_BYTES 176896
+LORA_API lora_status lora_shrink_noalloc(lora_dtype dtype, int T, int D, int r, int S,
+                                         int n_slices, const void* x, int64_t ldx,
+                                         const void* const* A, const int32_t* idx, float* buf,
+                                         int has_active, lora_stream_t stream);
+
 /* Static, human-readable name of a status. */
 LORA_API const char* lora_status_string(lora_status status);
 
