@@ -42,7 +42,8 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "gather_matmul_b200", "csrc", f)
-                  for f in ("bgmv.cu", "group.cu", "sgmv_tc.cu", "common.cuh")]
+                  for f in ("bgmv.cu", "bgmv_fused.cu", "group.cu", "sgmv_tc.cu", "common.cuh",
+                            "ptx.cuh")]
 
 
 # --------------------------------------------------------------------------
@@ -252,6 +253,18 @@ class DeviceSet:
         return sum(t.numel() * t.element_size() for t in ts)
 
 
+def fused(p):
+    from gather_matmul_b200 import ops
+    return (not p.segmented) and ops.bgmv_launches(W.TORCH_DTYPE[p.dtype], p.T, p.D, p.r, p.S,
+                                                   p.d_out) == 1
+
+
+def kernel_list(p):
+    if p.segmented:
+        return ["shrink", "expand"]
+    return ["fused"] if fused(p) else ["group", "shrink", "expand"]
+
+
 def step_calls(p, d, what="step"):
     """Enqueue one step (or one kernel of it) on the current stream."""
     from gather_matmul_b200 import ops
@@ -263,20 +276,24 @@ def step_calls(p, d, what="step"):
         if what in ("step", "expand"):
             ops.expand_segment(buf, d.B, d.ss, d.sa, d.y, d.meta, p.scale, y_col_off=p.col_off)
         return
-    if what in ("step", "group"):
+    if what in ("step", "fused"):
+        # the whole per-token path in one call (one launch when it fits);
+        # adapters and indices are never written by the preceding kernel here
+        ops.bgmv(d.x, d.A, d.B, d.idx, d.y, d.buf, d.meta, p.scale, y_col_off=p.col_off,
+                 pdl_early=True)
+        return
+    if what == "group":
         ops.group(d.idx, p.S, d.meta)
-    if what in ("step", "shrink"):
+    if what == "shrink":
         ops.shrink(d.x, d.A, d.buf, d.meta)
-    if what in ("step", "expand"):
+    if what == "expand":
         ops.expand(buf, d.B, d.y, d.meta, p.scale, y_col_off=p.col_off)
 
 
 def launches_per(p, what="step"):
-    if p.segmented:
-        per = {"shrink": 1, "expand": 1}
-    else:
-        per = {"group": 1, "shrink": 1, "expand": 1}
-    return sum(per.values()) if what == "step" else per.get(what, 0)
+    if what != "step":
+        return 1
+    return 2 if p.segmented else (1 if fused(p) else 3)
 
 
 class GraphRunner:
@@ -421,7 +438,13 @@ def measure_config(p, steps, warmup, stream, detail=False):
 
 def kernel_times(p, sets, stream, reps):
     out = {}
-    for what in (["group"] if not p.segmented else []) + ["shrink", "expand"]:
+    if not p.segmented and not fused(p):
+        # the group kernel must have run on each set before shrink / expand
+        for d in sets:
+            with torch.cuda.stream(stream):
+                step_calls(p, d, "group")
+        torch.cuda.synchronize()
+    for what in kernel_list(p):
         r = GraphRunner(p, sets, stream, what)
         plan = r.prepare(reps)
         with torch.cuda.stream(stream):
@@ -432,17 +455,27 @@ def kernel_times(p, sets, stream, reps):
     return out
 
 
-def roofline_entry(p, ktimes, peak, peak_kind):
+KERNEL_NAMES = {"fused": "bgmv_fused_kernel", "group": "group_kernel",
+                "shrink": "shrink_items_kernel", "expand": "expand_items_kernel"}
+SEG_KERNEL_NAMES = {"shrink": "sgmv_shrink", "expand": "sgmv_expand"}
+
+
+def kernel_bytes(p, what):
     by = algorithmic_bytes(p)
-    dom = max(("shrink", "expand"), key=lambda k: ktimes[k])
-    ach = by[dom] / ktimes[dom] / 1e9
-    name = {"shrink": "shrink_items_kernel", "expand": "expand_items_kernel"}[dom]
-    if p.segmented:
-        name = {"shrink": "sgmv_shrink", "expand": "sgmv_expand"}[dom]
+    if what == "fused":
+        return by["shrink"] + by["expand"]
+    return by[what]
+
+
+def roofline_entry(p, ktimes, peak, peak_kind):
+    dom = max((k for k in ktimes if k != "group"), key=lambda k: ktimes[k])
+    ach = kernel_bytes(p, dom) / ktimes[dom] / 1e9
+    name = (SEG_KERNEL_NAMES if p.segmented else KERNEL_NAMES)[dom]
     return {"bound": "hbm", "kernel": name, "achieved": round(ach, 1), "peak": peak,
             "peak_kind": peak_kind, "unit": "GB/s", "frac": round(ach / peak, 4),
             "traffic": profile_traffic(name),
-            "algorithmic_bytes": by[dom], "us_per_launch": round(ktimes[dom] * 1e6, 3)}
+            "algorithmic_bytes": kernel_bytes(p, dom),
+            "us_per_launch": round(ktimes[dom] * 1e6, 3)}
 
 
 def config_label(p):
@@ -500,8 +533,9 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": W.DTYPE_NAME[p.dtype], "data": "synthetic (seeded normal inputs, random adapters)",
         "config": {"workload": config_label(p),
-                   "step": "group-by-slot + shrink + expand" if not p.segmented
-                   else "segment shrink + expand",
+                   "step": ("segment shrink + expand" if p.segmented else
+                            "group-by-slot + shrink + expand in one fused launch" if fused(p)
+                            else "group-by-slot + shrink + expand (3 launches)"),
                    "l2": f"inputs larger than L2: {len(sets)} rotating input sets, "
                          f"{sum(s.nbytes() for s in sets) / 1e6:.0f} MB > {L2_BYTES / 1e6:.0f} MB",
                    "graph": "K steps replayed from CUDA graphs of up to 64 steps",
@@ -543,9 +577,9 @@ def detail_all(args, stream, peak, peak_kind):
                 "gbs_step": round(by["step"] / t / 1e9, 1),
                 "frac_step": round(by["step"] / t / 1e9 / peak, 4),
                 "kernel_us": {k: round(v * 1e6, 3) for k, v in kt.items()},
-                "kernel_gbs": {k: round(by[k] / v / 1e9, 1) for k, v in kt.items() if by.get(k)},
-                "kernel_frac": {k: round(by[k] / v / 1e9 / peak, 4) for k, v in kt.items()
-                                if by.get(k)},
+                "kernel_gbs": {k: round(kernel_bytes(p, k) / v / 1e9, 1) for k, v in kt.items()},
+                "kernel_frac": {k: round(kernel_bytes(p, k) / v / 1e9 / peak, 4)
+                                for k, v in kt.items()},
                 "tflops_step": round(fl / t / 1e12, 2),
                 "bytes": by,
             }
@@ -607,7 +641,7 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--steps", type=int, default=100000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -21,6 +21,7 @@ LORA_MAX_SLICES = 8
 LORA_MAX_SLOTS = 1024
 LORA_MAX_TOKENS = 1 << 22
 LORA_NOALLOC_MAX_TOKENS = 8192
+LORA_FLAG_PDL_EARLY = 1
 
 # Every symbol the header declares, with (restype, argtypes).
 _i32, _i64, _sz, _f32, _vp = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float, ctypes.c_void_p
@@ -36,6 +37,9 @@ SIGNATURES = {
                                    _i32, _vp, _i32, _vp, _sz, _vp]),
     "lora_expand_segment": (_i32, [_i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _vp,
                                    _i32, _f32, _vp, _i64, _vp, _i32, _vp, _sz, _vp]),
+    "lora_bgmv": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _i32, _vp, _vp, _f32,
+                         _vp, _i64, _vp, _vp, _vp, _i32, ctypes.c_uint, _vp, _sz, _vp]),
+    "lora_bgmv_launches": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp]),
     "lora_check_errors": (_i32, [_vp, _sz, _vp]),
     "lora_shrink_noalloc": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp,
                                    _vp, _i32, _vp]),

@@ -2,6 +2,7 @@
 // files.  Not part of the public interface.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -37,6 +38,35 @@ struct SegArgs {
   const int32_t* seg_adapter;
   int n_seg;
 };
+
+// Arguments of the fused per-token (BGMV) kernel: grouping, shrink and
+// expand of one batch in one launch.
+struct FusedArgs {
+  const void* x;
+  int64_t ldx;
+  const void* A[LORA_MAX_SLICES];
+  const void* B[LORA_MAX_SLICES];
+  int D_out[LORA_MAX_SLICES];
+  int64_t y_col_off[LORA_MAX_SLICES];
+  void* y;
+  int64_t ldy;
+  float* buf;               // [n_A][T][r], n_A = shared_A ? 1 : n_slices
+  const int32_t* idx;
+  int* bad_index;           // meta header counters
+  int* bad_meta;
+  int T, D, r, S, n_slices, shared_A;
+  float scale;
+  int pdl_early;            // A, B and idx may be read before the previous kernel ends
+};
+
+cudaError_t encode_tmap_2d(CUtensorMap* map, lora_dtype dt, const void* base, uint64_t inner,
+                           uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
+                           uint32_t box_outer, int swizzle_bytes);
+
+// Whether the fused kernel takes this shape (host-side, no CUDA calls).
+bool bgmv_fused_fits(int T, int D, int r, int n_slices, const int32_t* D_out);
+// Returns cudaErrorNotSupported when the shape does not fit the fused kernel.
+cudaError_t launch_bgmv_fused(lora_dtype dt, const FusedArgs& a, cudaStream_t st);
 
 size_t group_smem_bytes(int S);
 cudaError_t launch_group(int T, int S, const int32_t* idx, void* meta, cudaStream_t st);

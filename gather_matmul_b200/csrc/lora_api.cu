@@ -221,6 +221,72 @@ lora_status lora_expand_segment(lora_dtype dtype, int T, int r, int S, int n_sli
   return from_cuda(e);
 }
 
+static void fill_fused(FusedArgs& f, int T, int D, int r, int S, int n_slices, const void* x,
+                       int64_t ldx, const void* const* A, int shared_A, const void* const* B,
+                       const int32_t* D_out, float scale, void* y, int64_t ldy,
+                       const int64_t* y_col_off, float* buf, const int32_t* idx, void* meta,
+                       unsigned flags) {
+  f.x = x;
+  f.ldx = ldx;
+  for (int i = 0; i < n_slices; ++i) {
+    f.A[i] = A[shared_A ? 0 : i];
+    f.B[i] = B[i];
+    f.D_out[i] = D_out[i];
+    f.y_col_off[i] = y_col_off[i];
+  }
+  f.y = y;
+  f.ldy = ldy;
+  f.buf = buf;
+  f.idx = idx;
+  MetaHeader* h = static_cast<MetaHeader*>(meta);
+  f.bad_index = &h->bad_index;
+  f.bad_meta = &h->bad_meta;
+  f.T = T; f.D = D; f.r = r; f.S = S; f.n_slices = n_slices;
+  f.shared_A = shared_A ? 1 : 0;
+  f.scale = scale;
+  f.pdl_early = (flags & LORA_FLAG_PDL_EARLY) ? 1 : 0;
+}
+
+lora_status lora_bgmv(lora_dtype dtype, int T, int D, int r, int S, int n_slices, const void* x,
+                      int64_t ldx, const void* const* A, int shared_A, const void* const* B,
+                      const int32_t* D_out, float scale, void* y, int64_t ldy,
+                      const int64_t* y_col_off, float* buf, const int32_t* idx, int has_active,
+                      unsigned flags, void* meta, size_t meta_bytes, lora_stream_t stream) {
+  const int n_a = shared_A ? 1 : n_slices;
+  if (n_slices < 1 || n_slices > LORA_MAX_SLICES) return LORA_ERR_UNSUPPORTED;
+  if (A == nullptr && T > 0) return LORA_ERR_INVALID_ARG;
+  lora_status s = check_shrink(dtype, T, D, r, S, n_a, x, ldx, A, buf, meta, meta_bytes);
+  if (s != LORA_OK) return s;
+  s = check_expand(dtype, T, r, S, n_slices, buf, shared_A ? 0 : (int64_t)T * r, B, D_out, y, ldy,
+                   y_col_off, meta, meta_bytes);
+  if (s != LORA_OK) return s;
+  if (!has_active || T == 0) return LORA_OK;
+  if (idx == nullptr) return LORA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaGetLastError();
+  FusedArgs f = {};
+  fill_fused(f, T, D, r, S, n_slices, x, ldx, A, shared_A, B, D_out, scale, y, ldy, y_col_off,
+             buf, idx, meta, flags);
+  cudaError_t e = launch_bgmv_fused(dtype, f, st);
+  if (e != cudaErrorNotSupported) return from_cuda(e);
+  cudaGetLastError();
+  s = lora_group(T, S, idx, meta, meta_bytes, stream);
+  if (s != LORA_OK) return s;
+  s = lora_shrink(dtype, T, D, r, S, n_a, x, ldx, A, buf, 1, meta, meta_bytes, stream);
+  if (s != LORA_OK) return s;
+  return lora_expand(dtype, T, r, S, n_slices, buf, shared_A ? 0 : (int64_t)T * r, B, D_out,
+                     scale, y, ldy, y_col_off, 1, meta, meta_bytes, stream);
+}
+
+int lora_bgmv_launches(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
+                       const int32_t* D_out) {
+  if (dtype != LORA_F16 && dtype != LORA_BF16) return LORA_ERR_INVALID_ARG;
+  if (T < 0 || D <= 0 || n_slices < 1 || n_slices > LORA_MAX_SLICES || !rank_ok(r) || S < 1 ||
+      S > LORA_MAX_SLOTS || D_out == nullptr)
+    return LORA_ERR_UNSUPPORTED;
+  return bgmv_fused_fits(T, D, r, n_slices, D_out) ? 1 : 3;
+}
+
 lora_status lora_check_errors(void* meta, size_t meta_bytes, lora_stream_t stream) {
   if (meta == nullptr || meta_bytes < sizeof(MetaHeader)) return LORA_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;

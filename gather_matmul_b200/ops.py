@@ -124,6 +124,38 @@ def expand(buf: torch.Tensor, B: Sequence[torch.Tensor], y: torch.Tensor, meta: 
     return y
 
 
+def bgmv(x: torch.Tensor, A: Sequence[torch.Tensor], B: Sequence[torch.Tensor], idx: torch.Tensor,
+         y: torch.Tensor, buf: torch.Tensor, meta: torch.Tensor, scale: float = 1.0,
+         y_col_off=None, has_active: bool = True, pdl_early: bool = False, stream=None):
+    """group + shrink + expand of one batch in one call (one launch when the
+    shape fits the fused kernel).  A: one stack per slice of B, or a single
+    stack shared by every slice; buf: float32 [len(A), T, r] receives the
+    intermediate; y is updated in place.  pdl_early=True promises that A, B
+    and idx are not written by the kernel launched just before on the stream."""
+    T, D, ldx = _xinfo(x)
+    S, r, _ = A[0].shape
+    n = len(B)
+    shared = len(A) == 1 and n > 1
+    if not shared and len(A) != n:
+        raise ValueError("A must hold one stack per slice, or one shared stack")
+    _, ldy, _, _, _, d_out, off, _ = _expand_common(buf, B, y, y_col_off, None)
+    if idx.dtype != torch.int32 or not idx.is_contiguous():
+        raise TypeError("idx must be a contiguous int32 tensor")
+    flags = _lib.LORA_FLAG_PDL_EARLY if pdl_early else 0
+    _check("lora_bgmv", _lib.load().lora_bgmv(
+        _dtype(x), T, D, r, S, n, _ptr(x), ldx, _ptrs(A), int(shared), _ptrs(B), d_out,
+        ctypes.c_float(scale), _ptr(y), ldy, off, _ptr(buf), _ptr(idx), int(bool(has_active)),
+        flags, _ptr(meta), meta.numel(), _stream(stream)))
+    return y
+
+
+def bgmv_launches(dtype, T: int, D: int, r: int, S: int, d_out) -> int:
+    """Kernel launches bgmv() makes for this shape: 1 (fused) or 3."""
+    dt = _DT[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    arr = (ctypes.c_int32 * len(d_out))(*[int(v) for v in d_out])
+    return _lib.load().lora_bgmv_launches(dt, int(T), int(D), int(r), int(S), len(d_out), arr)
+
+
 def shrink_segment(x, A, seg_starts, seg_adapter, buf, meta, has_active=True, stream=None):
     """shrink() with adapters given by segments (int32 CSR starts [n+1], adapters [n])."""
     T, D, ldx = _xinfo(x)

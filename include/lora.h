@@ -160,6 +160,42 @@ LORA_API lora_status lora_expand(lora_dtype dtype, int T, int r, int S, int n_sl
                         size_t meta_bytes, lora_stream_t stream);
 
 /*
+ * Whole per-token (BGMV) LoRA of one batch in one call: lora_group, then
+ * lora_shrink, then lora_expand, with the same results (buf and y).  When the
+ * shape fits (T <= 4096 and the slot's tiles fit in shared memory) this is ONE
+ * kernel launch: each thread-block cluster owns one (slot, slice), finds its
+ * tokens itself, and keeps the fp32 intermediate on chip between the shrink
+ * and the expand (it is still written to buf).  Otherwise it runs the three
+ * launches.  Sources as for lora_shrink / lora_expand.
+ *
+ *   A, shared_A   shared_A = 0: A holds n_slices stacks (one per output slice);
+ *                 shared_A = 1: A[0] is one stack used by every slice.
+ *   buf           device fp32 [n_A, T, r], n_A = shared_A ? 1 : n_slices;
+ *                 receives the intermediate (required).
+ *   idx           device int32 [T] as for lora_group.
+ *   flags         LORA_FLAG_PDL_EARLY: A, B and idx are not written by the
+ *                 kernel launched just before this call on `stream`, so the
+ *                 call may read them before that kernel has finished
+ *                 (programmatic dependent launch); x and y are always read
+ *                 after it.  0: nothing is read before it finishes.
+ *   meta          workspace as for lora_group (its error counters are used;
+ *                 the three-launch path also keeps the grouping there).
+ *   Other arguments as for lora_shrink / lora_expand.
+ */
+#define LORA_FLAG_PDL_EARLY 1u
+LORA_API lora_status lora_bgmv(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
+                               const void* x, int64_t ldx, const void* const* A, int shared_A,
+                               const void* const* B, const int32_t* D_out, float scale, void* y,
+                               int64_t ldy, const int64_t* y_col_off, float* buf,
+                               const int32_t* idx, int has_active, unsigned flags, void* meta,
+                               size_t meta_bytes, lora_stream_t stream);
+
+/* Kernel launches lora_bgmv makes for this shape (1 fused, 3 otherwise), or a
+ * negative status for invalid sizes.  Host only; nothing is enqueued. */
+LORA_API int lora_bgmv_launches(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
+                                const int32_t* D_out);
+
+/*
  * SGMV shrink (segment-grouped, for prefill): contiguous runs of tokens share
  * one adapter.  Same result as lora_shrink with idx[t] = seg_adapter[s] for
  * seg_starts[s] <= t < seg_starts[s+1] ("Add multi-LoRA support", Limitations

@@ -65,6 +65,14 @@ class Dev:
         return self.y
 
 
+def run_bgmv(d: "Dev", pdl_early=False):
+    """The one-call per-token path (fused kernel when the shape fits)."""
+    p = d.p
+    ops.bgmv(d.x, d.A, d.B, d.idx, d.y, d.buf, d.meta, p.scale, y_col_off=p.col_off,
+             pdl_early=pdl_early)
+    return d.buf, d.y
+
+
 def problem_idx(p):
     if p.segmented:
         return oracle.segments_to_idx(p.T, p.seg_starts, p.seg_adapter)
