@@ -84,5 +84,11 @@ cudaError_t launch_shrink_segment_tc(lora_dtype dt, const ShrinkArgs& a, const S
                                      cudaStream_t st);
 cudaError_t launch_expand_segment_tc(lora_dtype dt, const ExpandArgs& a, const SegArgs& s,
                                      cudaStream_t st);
+// The same tensor-core kernels over the per-token grouping in meta (rows
+// gathered through the token permutation).
+cudaError_t launch_shrink_grouped_tc(lora_dtype dt, const ShrinkArgs& a, cudaStream_t st);
+cudaError_t launch_expand_grouped_tc(lora_dtype dt, const ExpandArgs& a, cudaStream_t st);
+// Whether the per-token calls use the tensor-core kernels for this shape.
+inline bool grouped_tc_preferred(int T, int r, int S) { return r >= 16 && T >= 16 * S; }
 
 }  // namespace lora

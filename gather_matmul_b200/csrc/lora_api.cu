@@ -127,6 +127,11 @@ lora_status lora_shrink(lora_dtype dtype, int T, int D, int r, int S, int n_slic
   a.T = T; a.D = D; a.r = r; a.S = S; a.n_slices = n_slices;
   a.meta = static_cast<const char*>(meta);
   cudaGetLastError();
+  if (grouped_tc_preferred(T, r, S)) {
+    cudaError_t e = launch_shrink_grouped_tc(dtype, a, (cudaStream_t)stream);
+    if (e != cudaErrorNotSupported) return from_cuda(e);
+    cudaGetLastError();
+  }
   return from_cuda(launch_shrink_items(dtype, a, max_items_tokens(T, S), (cudaStream_t)stream));
 }
 
@@ -161,6 +166,11 @@ lora_status lora_expand(lora_dtype dtype, int T, int r, int S, int n_slices,
   fill_expand(a, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, scale, y, ldy, y_col_off,
               meta);
   cudaGetLastError();
+  if (grouped_tc_preferred(T, r, S)) {
+    cudaError_t e = launch_expand_grouped_tc(dtype, a, (cudaStream_t)stream);
+    if (e != cudaErrorNotSupported) return from_cuda(e);
+    cudaGetLastError();
+  }
   return from_cuda(launch_expand_items(dtype, a, max_items_tokens(T, S), (cudaStream_t)stream));
 }
 

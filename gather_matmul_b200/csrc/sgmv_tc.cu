@@ -20,10 +20,11 @@
 //   One CTA per (tile, 128 output columns, slice).  The fp32 intermediate
 //   enters the tensor core as hi + lo of the input type after an exact
 //   power-of-two rescale per row (about 16 bits for bf16, 22 for fp16), two
-//   MMAs per K step into one fp32 accumulator.  The B tile arrives by TMA, the
-//   y rows of the tile by bulk copies into padded shared rows; the epilogue
-//   adds scale * acc with one round-to-nearest-even and writes y back with
-//   coalesced 16-byte stores.  Rows past the segment are never written.
+//   MMAs per K step into one fp32 accumulator.  The B tile arrives by TMA;
+//   each thread prefetches its row's y values into registers at the start
+//   (whole 32-byte sectors), so four CTAs fit per SM; the epilogue adds
+//   scale * acc with one round-to-nearest-even and stores from registers.
+//   Rows past the segment are never written.
 //
 // Every mbarrier wait is bounded (about one second); a timeout is counted in
 // the workspace and the kernel still releases its tensor memory and exits.
@@ -56,7 +57,8 @@ struct TileInfo {
 // access can leave the buffers even for malformed lists (those are counted
 // separately).  Warp-cooperative; every lane returns the same answer.
 __device__ bool find_tile(int tile, const int32_t* __restrict__ ss,
-                          const int32_t* __restrict__ sa, int n_seg, int T, TileInfo& ti) {
+                          const int32_t* __restrict__ sa, int n_seg, int T, TileInfo& ti,
+                          int implicit_slots) {
   const int lane = threadIdx.x & 31;
   int base = 0;
   for (int s0 = 0; s0 < n_seg; s0 += 32) {
@@ -83,7 +85,9 @@ __device__ bool find_tile(int tile, const int32_t* __restrict__ ss,
       ti.seg = s0 + l;
       ti.m0 = sa_l + (tile - base - excl) * kTM;
       ti.valid = min(kTM, sb_l - ti.m0);
-      ti.adapter = sa[s0 + l];
+      // per-token grouping: segment g is slot g, the last one holds the tokens
+      // without an adapter
+      ti.adapter = implicit_slots ? (s0 + l < implicit_slots ? s0 + l : -1) : sa[s0 + l];
       return true;
     }
     base += total;
@@ -106,6 +110,17 @@ __device__ void validate_segments(const int32_t* ss, const int32_t* sa, int n_se
   if (badi) atomicAdd(bad_index, badi);
 }
 
+// The per-token grouping in the workspace was built for (T, S): otherwise its
+// positions are not known to lie in this call's buffers, so nothing is done
+// and the error is counted once (the error counters head the workspace).
+__device__ bool grouped_meta_ok(int* counters, int T, int S) {
+  const MetaHeader* h = reinterpret_cast<const MetaHeader*>(counters);
+  if (h->T == T && h->S == S) return true;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0)
+    atomicAdd(&reinterpret_cast<MetaHeader*>(counters)->bad_meta, 1);
+  return false;
+}
+
 template <int SW>
 __device__ __forceinline__ int swz(int row, int chunk) {
   if constexpr (SW == 128) return chunk ^ (row & 7);
@@ -114,12 +129,15 @@ __device__ __forceinline__ int swz(int row, int chunk) {
 }
 
 struct ShrinkTCParams {
-  CUtensorMap tmX;                       // x as [T rows, D cols], box {64, 128}, 128B swizzle
+  CUtensorMap tmX;                       // x as [T rows, D cols], box {64, 128} (or {64, 1}
+                                         // for row gathers), 128B swizzle
   CUtensorMap tmA[LORA_MAX_SLICES];      // A_i as [S*r rows, D cols], box {64, r}, 128B swizzle
   const int32_t* seg_starts;
   const int32_t* seg_adapter;
   int n_seg;
   float* buf;
+  const int32_t* perm;                   // row p of a tile is token perm[p]; null = identity
+  int implicit_slots;                    // > 0: segment g is slot g (per-token grouping)
   int T, D, S, n_slices, KS;
   int* bad_index;
   int* bad_meta;
@@ -159,12 +177,14 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accbar + 1);
   int* sinfo = reinterpret_cast<int*>(tmem_slot + 4);
 
-  if (blockIdx.x == 0 && slice == 0)
+  if (blockIdx.x == 0 && slice == 0 && !P.implicit_slots)
     validate_segments(P.seg_starts, P.seg_adapter, P.n_seg, P.T, P.S, P.bad_index, P.bad_meta);
+  // grouping metadata must have been built for this call's sizes
+  const bool meta_ok = !P.implicit_slots || grouped_meta_ok(P.bad_index, P.T, P.S);
   if (warp == 0) {
     TileInfo ti;
-    const bool found =
-        find_tile(blockIdx.x / KS, P.seg_starts, P.seg_adapter, P.n_seg, P.T, ti);
+    const bool found = meta_ok && find_tile(blockIdx.x / KS, P.seg_starts, P.seg_adapter,
+                                            P.n_seg, P.T, ti, P.implicit_slots);
     if (lane == 0) {
       sinfo[0] = found ? 1 : 0;
       sinfo[1] = ti.m0;
@@ -176,9 +196,11 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   if (!sinfo[0]) return;                      // same for the whole cluster
   const int m0 = sinfo[1], valid = sinfo[2], adapter = sinfo[3];
   float* bufs = P.buf + (size_t)slice * P.T * R;
+  const int32_t* perm = P.perm;
+  auto token = [&](int p) { return perm ? perm[p] : p; };
   if (adapter < 0 || adapter >= P.S) {        // no adapter: zero rows (rank 0 writes them)
     if (kr == 0)
-      for (int e = tid; e < valid * R; e += kThreads) bufs[(size_t)(m0 + e / R) * R + e % R] = 0.f;
+      for (int e = tid; e < valid * R; e += kThreads) bufs[(size_t)token(m0 + e / R) * R + e % R] = 0.f;
     return;
   }
 
@@ -206,15 +228,37 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   const uint32_t tmem = *tmem_slot;
 
   bool ok = true;
-  if (tid == 0) {
-    const uint32_t sbase = ptx::smem_u32(smem);
-    auto issue = [&](int i, int s) {
+  const int ngroups = (valid + 3) / 4;        // 4-row gathers per stage (row indirection)
+  const uint32_t stage_bytes =
+      perm ? (uint32_t)(ngroups * 4 * 128 + L::kABytes) : (uint32_t)L::kStageBytes;
+  if (warp == 0) {
+    // producer warp: x tile (one 2-D tile, or up to 32 row gathers issued by
+    // the 32 lanes) and the adapter tile into stage s
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % kStages;
+      const uint32_t ph = (i / kStages) & 1;
+      if (i >= kStages) ok &= ptx::mbar_wait(&empty[s], ph ^ 1);   // MMAs of i - kStages done
       char* st = smem + (size_t)s * L::kStageBytes;
-      ptx::mbar_arrive_expect_tx(&full[s], L::kStageBytes);
-      ptx::tma_load_2d(st, &P.tmX, (kb0 + i) * kBK, m0, &full[s]);
-      ptx::tma_load_2d(st + L::kXBytes, &P.tmA[slice], (kb0 + i) * kBK, adapter * R, &full[s]);
-    };
-    for (int i = 0; i < kStages && i < nkb; ++i) issue(i, i);
+      const int kx = (kb0 + i) * kBK;
+      if (lane == 0) {
+        ptx::mbar_arrive_expect_tx(&full[s], stage_bytes);
+        ptx::tma_load_2d(st + L::kXBytes, &P.tmA[slice], kx, adapter * R, &full[s]);
+        if (!perm) ptx::tma_load_2d(st, &P.tmX, kx, m0, &full[s]);
+      }
+      __syncwarp();
+      if (perm && lane < ngroups) {
+        int rr[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int p = m0 + 4 * lane + j;
+          rr[j] = perm[p < m0 + valid ? p : m0];
+        }
+        ptx::tma_gather4(st + lane * 4 * 128, &P.tmX, kx, rr[0], rr[1], rr[2], rr[3], &full[s]);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // MMA issuer
+    const uint32_t sbase = ptx::smem_u32(smem);
     for (int i = 0; i < nkb; ++i) {
       const int s = i % kStages;
       const uint32_t ph = (i / kStages) & 1;
@@ -226,10 +270,6 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
         ptx::tc_mma_f16(tmem, ptx::umma_desc_kmajor(xa + k * 32, 128),
                         ptx::umma_desc_kmajor(aa + k * 32, 128), kIdesc, (i > 0 || k > 0) ? 1u : 0u);
       ptx::tc_commit(&empty[s]);              // stage s is free once these MMAs finish
-      if (i + kStages < nkb) {
-        ok &= ptx::mbar_wait(&empty[s], ph);
-        issue(i + kStages, s);
-      }
     }
     ptx::tc_commit(accbar);
   }
@@ -249,7 +289,7 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   const int m = warp * 32 + lane;
   if (KS == 1) {
     if (m < valid) {
-      float4* row = reinterpret_cast<float4*>(bufs + (size_t)(m0 + m) * R);
+      float4* row = reinterpret_cast<float4*>(bufs + (size_t)token(m0 + m) * R);
 #pragma unroll
       for (int q = 0; q < R / 4; ++q) row[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
@@ -266,7 +306,7 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
       const int mm = kr * rows + e / R, j = e % R;
       float s = 0.f;
       for (int q = 0; q < KS; ++q) s += cluster.map_shared_rank(part, q)[mm * L::kPitch + j];
-      if (mm < valid) bufs[(size_t)(m0 + mm) * R + j] = s;
+      if (mm < valid) bufs[(size_t)token(m0 + mm) * R + j] = s;
     }
     cluster.sync();                           // peers are done reading this CTA's partials
   }
@@ -287,6 +327,8 @@ struct ExpandTCParams {
   const int32_t* seg_starts;
   const int32_t* seg_adapter;
   int n_seg;
+  const int32_t* perm;                   // row p of a tile is token perm[p]; null = identity
+  int implicit_slots;                    // > 0: segment g is slot g (per-token grouping)
   int T, S, n_slices;
   float scale;
   int* bad_index;
@@ -298,14 +340,13 @@ struct ExpandSmem {
   static constexpr int kRowBytes = R * 2;                 // = swizzle width
   static constexpr int kBBytes = kNT * kRowBytes;
   static constexpr int kHBytes = kTM * kRowBytes;
-  static constexpr int kYPitch = kNT * 2 + 16;
   static constexpr size_t kOffB = 0, kOffHi = kBBytes, kOffLo = kOffHi + kHBytes,
-                          kOffY = kOffLo + kHBytes, kOffBar = kOffY + (size_t)kTM * kYPitch;
-  static constexpr size_t kTotal = kOffBar + 8 * 3 + 64 + 1024;
+                          kOffBar = kOffLo + kHBytes;
+  static constexpr size_t kTotal = kOffBar + 8 * 2 + 64 + 1024;
 };
 
 template <typename E, int R>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 4)
 sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   using L = ExpandSmem<R>;
   constexpr bool kBF = std::is_same<E, __nv_bfloat16>::value;
@@ -323,18 +364,18 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   char* sB = smem + L::kOffB;
   char* sHi = smem + L::kOffHi;
   char* sLo = smem + L::kOffLo;
-  char* sY = smem + L::kOffY;
   uint64_t* barB = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
-  uint64_t* barY = barB + 1;
-  uint64_t* accbar = barB + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barB + 3);
+  uint64_t* accbar = barB + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barB + 2);
   int* sinfo = reinterpret_cast<int*>(tmem_slot + 4);
 
-  if (blockIdx.x == 0 && blockIdx.y == 0 && slice == 0)
+  if (blockIdx.x == 0 && blockIdx.y == 0 && slice == 0 && !P.implicit_slots)
     validate_segments(P.seg_starts, P.seg_adapter, P.n_seg, P.T, P.S, P.bad_index, P.bad_meta);
+  const bool meta_ok = !P.implicit_slots || grouped_meta_ok(P.bad_index, P.T, P.S);
   if (warp == 0) {
     TileInfo ti;
-    const bool found = find_tile(blockIdx.x, P.seg_starts, P.seg_adapter, P.n_seg, P.T, ti);
+    const bool found = meta_ok && find_tile(blockIdx.x, P.seg_starts, P.seg_adapter, P.n_seg,
+                                            P.T, ti, P.implicit_slots);
     if (lane == 0) {
       sinfo[0] = found && ti.adapter >= 0 && ti.adapter < P.S ? 1 : 0;
       sinfo[1] = ti.m0;
@@ -349,7 +390,6 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
 
   if (tid == 0) {
     ptx::mbar_init(barB, 1);
-    ptx::mbar_init(barY, kThreads / 32);
     ptx::mbar_init(accbar, 1);
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&P.tmB[slice]);
@@ -363,44 +403,50 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // B tile (rows adapter*Dout + n0 ..) by TMA; y rows of the tile by bulk copies
+  // B tile (rows adapter*Dout + n0 ..) by TMA
   if (tid == 0) {
     ptx::mbar_arrive_expect_tx(barB, L::kBBytes);
     ptx::tma_load_2d(sB, &P.tmB[slice], 0, adapter * Dout + n0, barB);
   }
-  if (lane == 0) {
-    const int r0 = warp * 32, r1 = min(valid, r0 + 32);
-    ptx::mbar_arrive_expect_tx(barY, (uint32_t)(max(r1 - r0, 0) * nn * 2));
-    for (int mm = r0; mm < r1; ++mm)
-      ptx::bulk_g2s(sY + (size_t)mm * L::kYPitch, y + (size_t)(m0 + mm) * P.ldy, nn * 2, barY);
-  }
+  // this thread's row of y, prefetched into registers (one 32-byte sector per
+  // 16 columns) while the tile's operands are prepared
+  const int m = tid;
+  const int tok = m < valid ? (P.perm ? P.perm[m0 + m] : m0 + m) : 0;
+  E* yrow = y + (size_t)tok * P.ldy;
+  uint4 yv[kNT / 8];
+#pragma unroll
+  for (int c = 0; c < kNT / 8; ++c)
+    yv[c] = (m < valid && c * 8 < nn) ? *reinterpret_cast<const uint4*>(yrow + c * 8)
+                                      : make_uint4(0, 0, 0, 0);
 
   // row m's intermediate -> hi / lo operand rows (swizzled K-major), with an
   // exact power-of-two rescale 2^(7-e), e the exponent of max |buf| of the row
-  const int m = tid;
   float inv = 1.f;
   {
-    float v[R];
-    const float* brow = P.buf + (size_t)slice * P.buf_slice_stride + (size_t)(m0 + m) * R;
+    const float4* brow = reinterpret_cast<const float4*>(
+        P.buf + (size_t)slice * P.buf_slice_stride + (size_t)tok * R);
+    float mx = 0.f;                        // pass 1: the row's max |value|
 #pragma unroll
     for (int q = 0; q < R / 4; ++q) {
-      const float4 f = m < valid ? reinterpret_cast<const float4*>(brow)[q]
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-      v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+      const float4 f = m < valid ? brow[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+      mx = fmaxf(fmaxf(fmaxf(mx, fabsf(f.x)), fmaxf(fabsf(f.y), fabsf(f.z))), fabsf(f.w));
     }
-    float mx = 0.f;
-#pragma unroll
-    for (int j = 0; j < R; ++j) mx = fmaxf(mx, fabsf(v[j]));
     int e = ((__float_as_int(mx) >> 23) & 0xff) - 127;
     e = (mx > 0.f && e > -100 && e < 100) ? e : 0;
     const float sc = __int_as_float((127 - e + 7) << 23);
     inv = __int_as_float((127 + e - 7) << 23);
 #pragma unroll
-    for (int c = 0; c < R / 8; ++c) {
+    for (int c = 0; c < R / 8; ++c) {      // pass 2 (L1 hits): 8 values at a time
+      float4 f0 = make_float4(0.f, 0.f, 0.f, 0.f), f1 = f0;
+      if (m < valid) {
+        f0 = brow[2 * c];
+        f1 = brow[2 * c + 1];
+      }
+      const float x8[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
       uint16_t hi[8], lo[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const float x = v[c * 8 + u] * sc;
+        const float x = x8[u] * sc;
         hi[u] = Elem<E>::from_f32(x);
         lo[u] = Elem<E>::from_f32(x - Elem<E>::to_f32(hi[u]));
       }
@@ -427,32 +473,23 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
                       ptx::umma_desc_kmajor(bb + ks * 32, L::kRowBytes), kIdesc, 1u);
     ptx::tc_commit(accbar);
   }
-  ok &= ptx::mbar_wait(barY, 0);
   ok &= ptx::mbar_wait(accbar, 0);
   ptx::tc_fence_after();
 
-  // epilogue: TMEM lane m = this thread's row; 16 columns at a time
+  // epilogue: TMEM lane m = this thread's row; 16 columns at a time, one
+  // fp32 fma and one rounding per element, stores straight from registers
   for (int c = 0; c < kNT / 16; ++c) {
     uint32_t r[16];
     ptx::tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c * 16, r);
     ptx::tc_wait_ld();
     if (m < valid && c * 16 < nn) {
-      uint4* yp = reinterpret_cast<uint4*>(sY + (size_t)m * L::kYPitch + c * 32);
-      uint4 w[2] = {yp[0], yp[1]};
-      uint16_t* h = reinterpret_cast<uint16_t*>(w);
+      uint16_t* h = reinterpret_cast<uint16_t*>(&yv[2 * c]);
 #pragma unroll
       for (int u = 0; u < 16; ++u)
         h[u] = Elem<E>::from_f32(fmaf(P.scale, __uint_as_float(r[u]) * inv, Elem<E>::to_f32(h[u])));
-      yp[0] = w[0];
-      if (c * 16 + 8 < nn) yp[1] = w[1];
+      reinterpret_cast<uint4*>(yrow + c * 16)[0] = yv[2 * c];
+      if (c * 16 + 8 < nn) reinterpret_cast<uint4*>(yrow + c * 16)[1] = yv[2 * c + 1];
     }
-  }
-  __syncthreads();
-  const int cpr = nn / 8;                  // 16-byte chunks per row
-  for (int e = tid; e < valid * cpr; e += kThreads) {
-    const int mm = e / cpr, c = e % cpr;
-    *reinterpret_cast<uint4*>(y + (size_t)(m0 + mm) * P.ldy + c * 8) =
-        *reinterpret_cast<const uint4*>(sY + (size_t)mm * L::kYPitch + c * 16);
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -462,11 +499,12 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
 
 template <typename E, int R>
 cudaError_t shrink_tc_launch(const ShrinkArgs& a, const SegArgs& sg, lora_dtype dt,
-                             cudaStream_t st) {
+                             cudaStream_t st, const int32_t* perm, int implicit_slots) {
   ShrinkTCParams P;
   memset(&P, 0, sizeof(P));
+  // row gathers need a box one row high
   cudaError_t e = encode_tmap_2d(&P.tmX, dt, a.x, (uint64_t)a.D, (uint64_t)a.T,
-                                 (uint64_t)a.ldx * 2, kBK, kTM, 128);
+                                 (uint64_t)a.ldx * 2, kBK, perm ? 1 : kTM, 128);
   if (e != cudaSuccess) return e;
   for (int i = 0; i < a.n_slices; ++i) {
     e = encode_tmap_2d(&P.tmA[i], dt, a.A[i], (uint64_t)a.D, (uint64_t)a.S * R,
@@ -478,6 +516,8 @@ cudaError_t shrink_tc_launch(const ShrinkArgs& a, const SegArgs& sg, lora_dtype 
   P.seg_adapter = sg.seg_adapter;
   P.n_seg = sg.n_seg;
   P.buf = a.buf;
+  P.perm = perm;
+  P.implicit_slots = implicit_slots;
   P.T = a.T;
   P.D = a.D;
   P.S = a.S;
@@ -511,7 +551,7 @@ cudaError_t shrink_tc_launch(const ShrinkArgs& a, const SegArgs& sg, lora_dtype 
 
 template <typename E, int R>
 cudaError_t expand_tc_launch(const ExpandArgs& a, const SegArgs& sg, lora_dtype dt,
-                             cudaStream_t st) {
+                             cudaStream_t st, const int32_t* perm, int implicit_slots) {
   ExpandTCParams P;
   memset(&P, 0, sizeof(P));
   int max_nt = 0;
@@ -531,6 +571,8 @@ cudaError_t expand_tc_launch(const ExpandArgs& a, const SegArgs& sg, lora_dtype 
   P.seg_starts = sg.seg_starts;
   P.seg_adapter = sg.seg_adapter;
   P.n_seg = sg.n_seg;
+  P.perm = perm;
+  P.implicit_slots = implicit_slots;
   P.T = a.T;
   P.S = a.S;
   P.n_slices = a.n_slices;
@@ -549,33 +591,67 @@ cudaError_t expand_tc_launch(const ExpandArgs& a, const SegArgs& sg, lora_dtype 
 
 }  // namespace
 
-cudaError_t launch_shrink_segment_tc(lora_dtype dt, const ShrinkArgs& a, const SegArgs& s,
-                                     cudaStream_t st) {
+namespace {
+cudaError_t shrink_tc_any(lora_dtype dt, const ShrinkArgs& a, const SegArgs& s, cudaStream_t st,
+                          const int32_t* perm, int implicit) {
   if (a.D % 8 != 0 || a.ldx % 8 != 0) return cudaErrorNotSupported;
   const bool bf = dt == LORA_BF16;
   switch (a.r) {
-    case 16: return bf ? shrink_tc_launch<__nv_bfloat16, 16>(a, s, dt, st)
-                       : shrink_tc_launch<__half, 16>(a, s, dt, st);
-    case 32: return bf ? shrink_tc_launch<__nv_bfloat16, 32>(a, s, dt, st)
-                       : shrink_tc_launch<__half, 32>(a, s, dt, st);
-    case 64: return bf ? shrink_tc_launch<__nv_bfloat16, 64>(a, s, dt, st)
-                       : shrink_tc_launch<__half, 64>(a, s, dt, st);
+    case 16: return bf ? shrink_tc_launch<__nv_bfloat16, 16>(a, s, dt, st, perm, implicit)
+                       : shrink_tc_launch<__half, 16>(a, s, dt, st, perm, implicit);
+    case 32: return bf ? shrink_tc_launch<__nv_bfloat16, 32>(a, s, dt, st, perm, implicit)
+                       : shrink_tc_launch<__half, 32>(a, s, dt, st, perm, implicit);
+    case 64: return bf ? shrink_tc_launch<__nv_bfloat16, 64>(a, s, dt, st, perm, implicit)
+                       : shrink_tc_launch<__half, 64>(a, s, dt, st, perm, implicit);
     default: return cudaErrorNotSupported;     // rank 8: no M=128 tensor-core shape
   }
+}
+cudaError_t expand_tc_any(lora_dtype dt, const ExpandArgs& a, const SegArgs& s, cudaStream_t st,
+                          const int32_t* perm, int implicit) {
+  const bool bf = dt == LORA_BF16;
+  switch (a.r) {
+    case 16: return bf ? expand_tc_launch<__nv_bfloat16, 16>(a, s, dt, st, perm, implicit)
+                       : expand_tc_launch<__half, 16>(a, s, dt, st, perm, implicit);
+    case 32: return bf ? expand_tc_launch<__nv_bfloat16, 32>(a, s, dt, st, perm, implicit)
+                       : expand_tc_launch<__half, 32>(a, s, dt, st, perm, implicit);
+    case 64: return bf ? expand_tc_launch<__nv_bfloat16, 64>(a, s, dt, st, perm, implicit)
+                       : expand_tc_launch<__half, 64>(a, s, dt, st, perm, implicit);
+    default: return cudaErrorNotSupported;
+  }
+}
+// The per-token grouping as a segment list over the permuted token order:
+// slot g's tokens are positions [slot_off[g], slot_off[g+1]) of perm, and the
+// final range [slot_off[S], T) holds the tokens without an adapter.
+SegArgs grouped_segments(const char* meta, int T, int S) {
+  MetaLayout L(T, S);
+  SegArgs sg;
+  sg.seg_starts = reinterpret_cast<const int32_t*>(meta + L.off_slot);
+  sg.seg_adapter = nullptr;
+  sg.n_seg = S + 1;
+  return sg;
+}
+}  // namespace
+
+cudaError_t launch_shrink_segment_tc(lora_dtype dt, const ShrinkArgs& a, const SegArgs& s,
+                                     cudaStream_t st) {
+  return shrink_tc_any(dt, a, s, st, nullptr, 0);
 }
 
 cudaError_t launch_expand_segment_tc(lora_dtype dt, const ExpandArgs& a, const SegArgs& s,
                                      cudaStream_t st) {
-  const bool bf = dt == LORA_BF16;
-  switch (a.r) {
-    case 16: return bf ? expand_tc_launch<__nv_bfloat16, 16>(a, s, dt, st)
-                       : expand_tc_launch<__half, 16>(a, s, dt, st);
-    case 32: return bf ? expand_tc_launch<__nv_bfloat16, 32>(a, s, dt, st)
-                       : expand_tc_launch<__half, 32>(a, s, dt, st);
-    case 64: return bf ? expand_tc_launch<__nv_bfloat16, 64>(a, s, dt, st)
-                       : expand_tc_launch<__half, 64>(a, s, dt, st);
-    default: return cudaErrorNotSupported;
-  }
+  return expand_tc_any(dt, a, s, st, nullptr, 0);
+}
+
+cudaError_t launch_shrink_grouped_tc(lora_dtype dt, const ShrinkArgs& a, cudaStream_t st) {
+  MetaLayout L(a.T, a.S);
+  return shrink_tc_any(dt, a, grouped_segments(a.meta, a.T, a.S), st,
+                       reinterpret_cast<const int32_t*>(a.meta + L.off_perm), a.S);
+}
+
+cudaError_t launch_expand_grouped_tc(lora_dtype dt, const ExpandArgs& a, cudaStream_t st) {
+  MetaLayout L(a.T, a.S);
+  return expand_tc_any(dt, a, grouped_segments(a.meta, a.T, a.S), st,
+                       reinterpret_cast<const int32_t*>(a.meta + L.off_perm), a.S);
 }
 
 }  // namespace lora

@@ -68,10 +68,18 @@ def test_empty_batch():
     torch.cuda.synchronize()
 
 
-def test_unread_data_is_not_read():
+@pytest.mark.parametrize("shape", [dict(T=64, S=6, r=16, D=1032, d_out=(256, 64)),
+                                   dict(T=160, S=5, r=32, D=2056, d_out=(384, 136))],
+                         ids=["cuda-core-items", "tensor-core-grouped"])
+def test_unread_data_is_not_read(shape):
     # x rows and y rows of -1 tokens, and the weights of slots nobody uses,
     # are poisoned with NaN; results must not change.
-    p = _p(seed=9, T=64, S=6, kind="uniform_neg")
+    p = _p(seed=9, kind="uniform_neg", **shape)
+    if shape["S"] == 5:   # leave slot 3 unused
+        idx = p.idx.copy()
+        idx[idx == 3] = 2
+        import dataclasses
+        p = dataclasses.replace(p, idx=idx)
     used = set(int(v) for v in p.idx if v >= 0)
     unused = [g for g in range(p.S) if g not in used]
     nan_bits = np.uint16(0x7FC0 if p.dtype == W.BF16 else 0x7E00)
