@@ -154,8 +154,12 @@ struct ShrinkSmem {
   static constexpr size_t kTotal = kBar + 8 * (2 * kStages + 1) + 64 + 1024;
 };
 
+// warps 0-3: loads (one per SM sub-partition, so small gathers issue four-wide),
+// then the epilogue on TMEM lane quadrant = warp; warp 4: MMA issue.
+constexpr int kShrThreads = 160;
+
 template <typename E, int R>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kShrThreads, 2)
 sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   using L = ShrinkSmem<R>;
   constexpr int kStages = L::kStages;
@@ -200,7 +204,7 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   auto token = [&](int p) { return perm ? perm[p] : p; };
   if (adapter < 0 || adapter >= P.S) {        // no adapter: zero rows (rank 0 writes them)
     if (kr == 0)
-      for (int e = tid; e < valid * R; e += kThreads) bufs[(size_t)token(m0 + e / R) * R + e % R] = 0.f;
+      for (int e = tid; e < valid * R; e += kShrThreads) bufs[(size_t)token(m0 + e / R) * R + e % R] = 0.f;
     return;
   }
 
@@ -210,15 +214,15 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      ptx::mbar_init(&full[s], 1);
-      ptx::mbar_init(&empty[s], 1);
+      ptx::mbar_init(&full[s], 4);           // one arrival per load warp
+      ptx::mbar_init(&empty[s], 1);          // tcgen05.commit
     }
     ptx::mbar_init(accbar, 1);
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&P.tmX);
     ptx::prefetch_tensormap(&P.tmA[slice]);
   }
-  if (warp == 0) {
+  if (warp == 4) {
     ptx::tmem_alloc(tmem_slot, kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -231,33 +235,39 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   const int ngroups = (valid + 3) / 4;        // 4-row gathers per stage (row indirection)
   const uint32_t stage_bytes =
       perm ? (uint32_t)(ngroups * 4 * 128 + L::kABytes) : (uint32_t)L::kStageBytes;
-  if (warp == 0) {
-    // producer warp: x tile (one 2-D tile, or up to 32 row gathers issued by
-    // the 32 lanes) and the adapter tile into stage s
+  if (warp < 4) {
+    // load warps: the adapter tile and the x tile (one 2-D tile, or up to 32
+    // four-row gathers, gather g issued by warp g % 4, lane g / 4)
     for (int i = 0; i < nkb; ++i) {
       const int s = i % kStages;
       const uint32_t ph = (i / kStages) & 1;
       if (i >= kStages) ok &= ptx::mbar_wait(&empty[s], ph ^ 1);   // MMAs of i - kStages done
       char* st = smem + (size_t)s * L::kStageBytes;
       const int kx = (kb0 + i) * kBK;
+      const int mine = perm ? max((ngroups - warp + 3) / 4, 0) : 0;
       if (lane == 0) {
-        ptx::mbar_arrive_expect_tx(&full[s], stage_bytes);
-        ptx::tma_load_2d(st + L::kXBytes, &P.tmA[slice], kx, adapter * R, &full[s]);
-        if (!perm) ptx::tma_load_2d(st, &P.tmX, kx, m0, &full[s]);
+        uint32_t bytes = (uint32_t)(mine * 512);
+        if (warp == 0) bytes += (uint32_t)L::kABytes + (perm ? 0u : (uint32_t)L::kXBytes);
+        ptx::mbar_arrive_expect_tx(&full[s], bytes);
+        if (warp == 0) {
+          ptx::tma_load_2d(st + L::kXBytes, &P.tmA[slice], kx, adapter * R, &full[s]);
+          if (!perm) ptx::tma_load_2d(st, &P.tmX, kx, m0, &full[s]);
+        }
       }
       __syncwarp();
-      if (perm && lane < ngroups) {
+      const int g = warp + 4 * lane;
+      if (perm && g < ngroups) {
         int rr[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int p = m0 + 4 * lane + j;
+          const int p = m0 + 4 * g + j;
           rr[j] = perm[p < m0 + valid ? p : m0];
         }
-        ptx::tma_gather4(st + lane * 4 * 128, &P.tmX, kx, rr[0], rr[1], rr[2], rr[3], &full[s]);
+        ptx::tma_gather4(st + g * 4 * 128, &P.tmX, kx, rr[0], rr[1], rr[2], rr[3], &full[s]);
       }
     }
-  } else if (warp == 1 && lane == 0) {
-    // MMA issuer
+  } else if (lane == 0) {
+    // MMA issuer (warp 4)
     const uint32_t sbase = ptx::smem_u32(smem);
     for (int i = 0; i < nkb; ++i) {
       const int s = i % kStages;
@@ -276,48 +286,59 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   ok &= ptx::mbar_wait(accbar, 0);
   ptx::tc_fence_after();
 
-  // accumulator row m = 32 * warp + lane, r fp32 columns
-  float v[R];
-#pragma unroll
-  for (int c = 0; c < R / 16; ++c) {
-    uint32_t r[16];
-    ptx::tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c * 16, r);
-    ptx::tc_wait_ld();
-#pragma unroll
-    for (int u = 0; u < 16; ++u) v[c * 16 + u] = __uint_as_float(r[u]);
-  }
+  // accumulator row m = 32 * warp + lane (warps 0-3), r fp32 columns
+  const bool has_row = warp < 4;
   const int m = warp * 32 + lane;
+  float v[R];
+  if (has_row) {
+#pragma unroll
+    for (int c = 0; c < R / 16; ++c) {
+      uint32_t r[16];
+      ptx::tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c * 16, r);
+      ptx::tc_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[c * 16 + u] = __uint_as_float(r[u]);
+    }
+  }
   if (KS == 1) {
-    if (m < valid) {
+    if (has_row && m < valid) {
       float4* row = reinterpret_cast<float4*>(bufs + (size_t)token(m0 + m) * R);
 #pragma unroll
       for (int q = 0; q < R / 4; ++q) row[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
   } else {
-    // every stage is drained (accbar): reuse the stage memory for partials
-    float* part = reinterpret_cast<float*>(smem);
+    // Split-K sum.  Row m belongs to rank m / rows; every rank pushes its
+    // partial row into slot [kr] of the owner's receive area (the owner's
+    // drained stage memory), then each owner adds its KS slots in rank order.
+    const int rows = kTM / KS;
+    cluster.barrier_arrive();                 // this CTA's MMAs and stages are done...
+    cluster.barrier_wait();                   // ...and so are every peer's
+    float* recv = reinterpret_cast<float*>(smem);
+    if (has_row) {
+      float* dst = cluster.map_shared_rank(recv, m / rows) + (size_t)(kr * rows + m % rows) * L::kPitch;
 #pragma unroll
-    for (int q = 0; q < R / 4; ++q)
-      *reinterpret_cast<float4*>(part + m * L::kPitch + 4 * q) =
-          make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-    cluster.sync();
-    const int rows = kTM / KS;                // rank kr sums rows [kr*rows, (kr+1)*rows)
-    for (int e = tid; e < rows * R; e += kThreads) {
-      const int mm = kr * rows + e / R, j = e % R;
-      float s = 0.f;
-      for (int q = 0; q < KS; ++q) s += cluster.map_shared_rank(part, q)[mm * L::kPitch + j];
-      if (mm < valid) bufs[(size_t)token(m0 + mm) * R + j] = s;
+      for (int q = 0; q < R / 4; ++q)
+        reinterpret_cast<float4*>(dst)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
-    cluster.sync();                           // peers are done reading this CTA's partials
+    cluster.sync();                           // every partial has arrived
+    for (int e = tid; e < rows * R; e += kShrThreads) {
+      const int lm = e / R, j = e % R;
+      float sum = 0.f;
+      for (int q = 0; q < KS; ++q) sum += recv[(size_t)(q * rows + lm) * L::kPitch + j];
+      const int mm = kr * rows + lm;
+      if (mm < valid) bufs[(size_t)token(m0 + mm) * R + j] = sum;
+    }
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 0) ptx::tmem_dealloc(tmem, kTmemCols);
+  if (warp == 4) ptx::tmem_dealloc(tmem, kTmemCols);
   if (!ok && tid == 0) atomicAdd(P.bad_meta, 1);
 }
 
 struct ExpandTCParams {
   CUtensorMap tmB[LORA_MAX_SLICES];      // B_i as [S*D_out_i rows, r cols], box {r, 128}
+  CUtensorMap tmY;                       // y as [T rows, ldy cols], box {64, 128}, 128B swizzle
+  CUtensorMap tmYg;                      // y, box {64, 1}: 4-row gathers
   const float* buf;
   int64_t buf_slice_stride;
   void* y;
@@ -330,6 +351,7 @@ struct ExpandTCParams {
   const int32_t* perm;                   // row p of a tile is token perm[p]; null = identity
   int implicit_slots;                    // > 0: segment g is slot g (per-token grouping)
   int T, S, n_slices;
+  int NJ, n_chunks;                      // each CTA walks NJ consecutive 128-column tiles
   float scale;
   int* bad_index;
   int* bad_meta;
@@ -337,26 +359,39 @@ struct ExpandTCParams {
 
 template <int R>
 struct ExpandSmem {
-  static constexpr int kRowBytes = R * 2;                 // = swizzle width
+  static constexpr int kYS = 3;                           // {B tile, y tile} ring stages
+  static constexpr int kRowBytes = R * 2;                 // = swizzle width of the operands
   static constexpr int kBBytes = kNT * kRowBytes;
   static constexpr int kHBytes = kTM * kRowBytes;
-  static constexpr size_t kOffB = 0, kOffHi = kBBytes, kOffLo = kOffHi + kHBytes,
-                          kOffBar = kOffLo + kHBytes;
-  static constexpr size_t kTotal = kOffBar + 8 * 2 + 64 + 1024;
+  static constexpr int kYHalf = kTM * 128;                // 64 columns x 128 rows, 128B swizzle
+  static constexpr int kYBytes = 2 * kYHalf;
+  static constexpr size_t kOffB = 0;
+  static constexpr size_t kOffHi = kOffB + (size_t)kYS * kBBytes;
+  static constexpr size_t kOffLo = kOffHi + kHBytes;
+  static constexpr size_t kOffY = kOffLo + kHBytes;
+  static constexpr size_t kOffBar = kOffY + (size_t)kYS * kYBytes;
+  static constexpr size_t kTotal = kOffBar + 8 * (2 * kYS + 5) + 64 + 1024;
 };
 
+// warps 0-3: epilogue (TMEM lane quadrant = warp), warps 4-7: loads (one per
+// SM sub-partition, so small copies issue four-wide), warp 8: MMA issue.
+constexpr int kExpThreads = 288;
+
 template <typename E, int R>
-__global__ void __launch_bounds__(kThreads, 4)
+__global__ void __launch_bounds__(kExpThreads, 1)
 sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   using L = ExpandSmem<R>;
+  constexpr int kYS = L::kYS;
   constexpr bool kBF = std::is_same<E, __nv_bfloat16>::value;
   constexpr uint32_t kIdesc = ptx::umma_idesc_f16(kBF, kTM, kNT);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int slice = blockIdx.z;
+  const int slice = blockIdx.y;
   const int Dout = P.D_out[slice];
-  const int n0 = blockIdx.y * kNT;
-  if (n0 >= Dout) return;
-  const int nn = min(kNT, Dout - n0);
+  const int ntiles = (Dout + kNT - 1) / kNT;
+  const int chunk = blockIdx.x % P.n_chunks;
+  const int j0 = chunk * P.NJ, j1 = min(ntiles, j0 + P.NJ);
+  if (j0 >= j1) return;
+  const int nj = j1 - j0;
 
   extern __shared__ char smem_raw[];
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -364,18 +399,22 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   char* sB = smem + L::kOffB;
   char* sHi = smem + L::kOffHi;
   char* sLo = smem + L::kOffLo;
-  uint64_t* barB = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
-  uint64_t* accbar = barB + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barB + 2);
+  char* sY = smem + L::kOffY;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* empty = full + kYS;
+  uint64_t* accfull = empty + kYS;       // [2]
+  uint64_t* accempty = accfull + 2;      // [2]
+  uint64_t* hilo = accempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(hilo + 1);
   int* sinfo = reinterpret_cast<int*>(tmem_slot + 4);
 
-  if (blockIdx.x == 0 && blockIdx.y == 0 && slice == 0 && !P.implicit_slots)
+  if (blockIdx.x == 0 && slice == 0 && !P.implicit_slots)
     validate_segments(P.seg_starts, P.seg_adapter, P.n_seg, P.T, P.S, P.bad_index, P.bad_meta);
   const bool meta_ok = !P.implicit_slots || grouped_meta_ok(P.bad_index, P.T, P.S);
   if (warp == 0) {
     TileInfo ti;
-    const bool found = meta_ok && find_tile(blockIdx.x, P.seg_starts, P.seg_adapter, P.n_seg,
-                                            P.T, ti, P.implicit_slots);
+    const bool found = meta_ok && find_tile(blockIdx.x / P.n_chunks, P.seg_starts, P.seg_adapter,
+                                            P.n_seg, P.T, ti, P.implicit_slots);
     if (lane == 0) {
       sinfo[0] = found && ti.adapter >= 0 && ti.adapter < P.S ? 1 : 0;
       sinfo[1] = ti.m0;
@@ -386,115 +425,211 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   __syncthreads();
   if (!sinfo[0]) return;                 // no tile, or rows without an adapter: untouched
   const int m0 = sinfo[1], valid = sinfo[2], adapter = sinfo[3];
-  E* y = static_cast<E*>(P.y) + P.y_col_off[slice] + n0;
+  const int64_t ycol0 = P.y_col_off[slice];
+  E* ycol = static_cast<E*>(P.y) + ycol0;
+  // whole 128-row tile of consecutive tokens: y moves as 2-D TMA tiles
+  const bool tiled = P.perm == nullptr && valid == kTM;
 
   if (tid == 0) {
-    ptx::mbar_init(barB, 1);
-    ptx::mbar_init(accbar, 1);
+    for (int s = 0; s < kYS; ++s) {
+      ptx::mbar_init(&full[s], 4);       // one arrival per load warp
+      ptx::mbar_init(&empty[s], 4);      // one arrival per epilogue warp
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(&accfull[a], 1);
+      ptx::mbar_init(&accempty[a], 4);
+    }
+    ptx::mbar_init(hilo, 4);
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&P.tmB[slice]);
+    ptx::prefetch_tensormap(tiled ? &P.tmY : &P.tmYg);
   }
-  if (warp == 0) {
-    ptx::tmem_alloc(tmem_slot, kNT);
+  if (warp == 8) {
+    ptx::tmem_alloc(tmem_slot, 2 * kNT);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  // B tile (rows adapter*Dout + n0 ..) by TMA
-  if (tid == 0) {
-    ptx::mbar_arrive_expect_tx(barB, L::kBBytes);
-    ptx::tma_load_2d(sB, &P.tmB[slice], 0, adapter * Dout + n0, barB);
-  }
-  // this thread's row of y, prefetched into registers (one 32-byte sector per
-  // 16 columns) while the tile's operands are prepared
-  const int m = tid;
-  const int tok = m < valid ? (P.perm ? P.perm[m0 + m] : m0 + m) : 0;
-  E* yrow = y + (size_t)tok * P.ldy;
-  uint4 yv[kNT / 8];
-#pragma unroll
-  for (int c = 0; c < kNT / 8; ++c)
-    yv[c] = (m < valid && c * 8 < nn) ? *reinterpret_cast<const uint4*>(yrow + c * 8)
-                                      : make_uint4(0, 0, 0, 0);
-
-  // row m's intermediate -> hi / lo operand rows (swizzled K-major), with an
-  // exact power-of-two rescale 2^(7-e), e the exponent of max |buf| of the row
-  float inv = 1.f;
-  {
-    const float4* brow = reinterpret_cast<const float4*>(
-        P.buf + (size_t)slice * P.buf_slice_stride + (size_t)tok * R);
-    float mx = 0.f;                        // pass 1: the row's max |value|
-#pragma unroll
-    for (int q = 0; q < R / 4; ++q) {
-      const float4 f = m < valid ? brow[q] : make_float4(0.f, 0.f, 0.f, 0.f);
-      mx = fmaxf(fmaxf(fmaxf(mx, fabsf(f.x)), fmaxf(fabsf(f.y), fabsf(f.z))), fabsf(f.w));
-    }
-    int e = ((__float_as_int(mx) >> 23) & 0xff) - 127;
-    e = (mx > 0.f && e > -100 && e < 100) ? e : 0;
-    const float sc = __int_as_float((127 - e + 7) << 23);
-    inv = __int_as_float((127 + e - 7) << 23);
-#pragma unroll
-    for (int c = 0; c < R / 8; ++c) {      // pass 2 (L1 hits): 8 values at a time
-      float4 f0 = make_float4(0.f, 0.f, 0.f, 0.f), f1 = f0;
-      if (m < valid) {
-        f0 = brow[2 * c];
-        f1 = brow[2 * c + 1];
-      }
-      const float x8[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-      uint16_t hi[8], lo[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float x = x8[u] * sc;
-        hi[u] = Elem<E>::from_f32(x);
-        lo[u] = Elem<E>::from_f32(x - Elem<E>::to_f32(hi[u]));
-      }
-      const int off = m * L::kRowBytes + swz<L::kRowBytes>(m, c) * 16;
-      *reinterpret_cast<uint4*>(sHi + off) = *reinterpret_cast<const uint4*>(hi);
-      *reinterpret_cast<uint4*>(sLo + off) = *reinterpret_cast<const uint4*>(lo);
-    }
-  }
-  ptx::fence_proxy_async_smem();           // generic writes -> tensor-core operand reads
-  __syncthreads();
-
   bool ok = true;
-  if (tid == 0) {
-    ok &= ptx::mbar_wait(barB, 0);
-    ptx::tc_fence_after();
-    const uint32_t hb = ptx::smem_u32(sHi), lb = ptx::smem_u32(sLo), bb = ptx::smem_u32(sB);
-#pragma unroll
-    for (int ks = 0; ks < R / 16; ++ks)
-      ptx::tc_mma_f16(tmem, ptx::umma_desc_kmajor(hb + ks * 32, L::kRowBytes),
-                      ptx::umma_desc_kmajor(bb + ks * 32, L::kRowBytes), kIdesc, ks > 0 ? 1u : 0u);
-#pragma unroll
-    for (int ks = 0; ks < R / 16; ++ks)
-      ptx::tc_mma_f16(tmem, ptx::umma_desc_kmajor(lb + ks * 32, L::kRowBytes),
-                      ptx::umma_desc_kmajor(bb + ks * 32, L::kRowBytes), kIdesc, 1u);
-    ptx::tc_commit(accbar);
-  }
-  ok &= ptx::mbar_wait(accbar, 0);
-  ptx::tc_fence_after();
 
-  // epilogue: TMEM lane m = this thread's row; 16 columns at a time, one
-  // fp32 fma and one rounding per element, stores straight from registers
-  for (int c = 0; c < kNT / 16; ++c) {
-    uint32_t r[16];
-    ptx::tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c * 16, r);
-    ptx::tc_wait_ld();
-    if (m < valid && c * 16 < nn) {
-      uint16_t* h = reinterpret_cast<uint16_t*>(&yv[2 * c]);
+  if (warp >= 4 && warp < 8) {
+    // ---- loads: B tile and y tile of n-tile j into stage j % kYS
+    const int pw = warp - 4;
+    const int ngroups = (valid + 3) / 4;
+    for (int j = 0; j < nj; ++j) {
+      const int s = j % kYS;
+      if (j >= kYS) ok &= ptx::mbar_wait(&empty[s], ((j / kYS) - 1) & 1);
+      const int n0 = (j0 + j) * kNT;
+      char* ys = sY + (size_t)s * L::kYBytes;
+      // ops of this n-tile: 2 y halves x ngroups 4-row gathers, dealt out over
+      // the four load warps (op o -> warp o % 4, lane o / 4)
+      int my_ops = 0;
+      if (!tiled)
+        for (int o = pw; o < 2 * ngroups; o += 4) ++my_ops;
+      const uint32_t bytes = (uint32_t)(my_ops * 512) +
+                             (pw == 0 ? (uint32_t)L::kBBytes + (tiled ? (uint32_t)L::kYBytes : 0u) : 0u);
+      if (lane == 0) {
+        ptx::mbar_arrive_expect_tx(&full[s], bytes);
+        if (pw == 0) {
+          ptx::tma_load_2d(sB + (size_t)s * L::kBBytes, &P.tmB[slice], 0, adapter * Dout + n0,
+                           &full[s]);
+          if (tiled) {
+            ptx::tma_load_2d(ys, &P.tmY, (int)(ycol0 + n0), m0, &full[s]);
+            ptx::tma_load_2d(ys + L::kYHalf, &P.tmY, (int)(ycol0 + n0 + 64), m0, &full[s]);
+          }
+        }
+      }
+      __syncwarp();
+      if (!tiled) {
+        for (int o = pw + 4 * lane; o < 2 * ngroups; o += 128) {
+          const int g = o >> 1, h = o & 1;
+          int rr[4];
 #pragma unroll
-      for (int u = 0; u < 16; ++u)
-        h[u] = Elem<E>::from_f32(fmaf(P.scale, __uint_as_float(r[u]) * inv, Elem<E>::to_f32(h[u])));
-      reinterpret_cast<uint4*>(yrow + c * 16)[0] = yv[2 * c];
-      if (c * 16 + 8 < nn) reinterpret_cast<uint4*>(yrow + c * 16)[1] = yv[2 * c + 1];
+          for (int q = 0; q < 4; ++q) {
+            const int mm = 4 * g + q < valid ? 4 * g + q : 0;
+            rr[q] = P.perm ? P.perm[m0 + mm] : m0 + mm;
+          }
+          ptx::tma_gather4(ys + h * L::kYHalf + g * 512, &P.tmYg, (int)(ycol0 + n0 + 64 * h),
+                           rr[0], rr[1], rr[2], rr[3], &full[s]);
+        }
+      }
     }
+  } else if (warp == 8) {
+    // ---- MMA issue: acc[j & 1] = hi . B^T + lo . B^T
+    if (lane == 0) {
+      ok &= ptx::mbar_wait(hilo, 0);
+      const uint32_t hb = ptx::smem_u32(sHi), lb = ptx::smem_u32(sLo);
+      for (int j = 0; j < nj; ++j) {
+        const int s = j % kYS, a = j & 1;
+        ok &= ptx::mbar_wait(&full[s], (j / kYS) & 1);
+        if (j >= 2) ok &= ptx::mbar_wait(&accempty[a], ((j / 2) - 1) & 1);
+        ptx::tc_fence_after();
+        const uint32_t bb = ptx::smem_u32(sB + (size_t)s * L::kBBytes);
+        const uint32_t acc = tmem + a * kNT;
+#pragma unroll
+        for (int ks = 0; ks < R / 16; ++ks)
+          ptx::tc_mma_f16(acc, ptx::umma_desc_kmajor(hb + ks * 32, L::kRowBytes),
+                          ptx::umma_desc_kmajor(bb + ks * 32, L::kRowBytes), kIdesc,
+                          ks > 0 ? 1u : 0u);
+#pragma unroll
+        for (int ks = 0; ks < R / 16; ++ks)
+          ptx::tc_mma_f16(acc, ptx::umma_desc_kmajor(lb + ks * 32, L::kRowBytes),
+                          ptx::umma_desc_kmajor(bb + ks * 32, L::kRowBytes), kIdesc, 1u);
+        ptx::tc_commit(&accfull[a]);
+      }
+    }
+  } else {
+    // ---- epilogue warps 0-3: row m = TMEM lane 32 * warp + lane
+    const int m = warp * 32 + lane;
+    const int tok = m < valid ? (P.perm ? P.perm[m0 + m] : m0 + m) : 0;
+    // row m's intermediate -> hi / lo operand rows (swizzled K-major), after an
+    // exact power-of-two rescale 2^(7-e), e the exponent of max |buf| of the row
+    float inv = 1.f;
+    {
+      const float4* brow = reinterpret_cast<const float4*>(
+          P.buf + (size_t)slice * P.buf_slice_stride + (size_t)tok * R);
+      float mx = 0.f;
+#pragma unroll
+      for (int q = 0; q < R / 4; ++q) {
+        const float4 f = m < valid ? brow[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+        mx = fmaxf(fmaxf(fmaxf(mx, fabsf(f.x)), fmaxf(fabsf(f.y), fabsf(f.z))), fabsf(f.w));
+      }
+      int e = ((__float_as_int(mx) >> 23) & 0xff) - 127;
+      e = (mx > 0.f && e > -100 && e < 100) ? e : 0;
+      const float sc = __int_as_float((127 - e + 7) << 23);
+      inv = __int_as_float((127 + e - 7) << 23);
+#pragma unroll
+      for (int c = 0; c < R / 8; ++c) {
+        float4 f0 = make_float4(0.f, 0.f, 0.f, 0.f), f1 = f0;
+        if (m < valid) {
+          f0 = brow[2 * c];
+          f1 = brow[2 * c + 1];
+        }
+        const float x8[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+        uint16_t hi[8], lo[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float xv = x8[u] * sc;
+          hi[u] = Elem<E>::from_f32(xv);
+          lo[u] = Elem<E>::from_f32(xv - Elem<E>::to_f32(hi[u]));
+        }
+        const int off = m * L::kRowBytes + swz<L::kRowBytes>(m, c) * 16;
+        *reinterpret_cast<uint4*>(sHi + off) = *reinterpret_cast<const uint4*>(hi);
+        *reinterpret_cast<uint4*>(sLo + off) = *reinterpret_cast<const uint4*>(lo);
+      }
+    }
+    ptx::fence_proxy_async_smem();       // generic writes -> tensor-core operand reads
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(hilo);
+
+    for (int j = 0; j < nj; ++j) {
+      const int s = j % kYS, a = j & 1;
+      const int n0 = (j0 + j) * kNT, nn = min(kNT, Dout - n0);
+      ok &= ptx::mbar_wait(&accfull[a], (j / 2) & 1);
+      ok &= ptx::mbar_wait(&full[s], (j / kYS) & 1);
+      ptx::tc_fence_after();
+      char* ys = sY + (size_t)s * L::kYBytes;
+      // y tile layout: two 64-column halves, 128-byte rows, 16-byte chunk q of
+      // a row at position q ^ (row & 7)
+      for (int c = 0; c < kNT / 16; ++c) {
+        uint32_t r[16];
+        ptx::tc_ld16(tmem + a * kNT + ((uint32_t)(warp * 32) << 16) + c * 16, r);
+        ptx::tc_wait_ld();
+        if (m < valid) {
+          char* hbase = ys + (c >> 2) * L::kYHalf + m * 128;
+          uint4* p0 = reinterpret_cast<uint4*>(hbase + ((((2 * c) & 7)) ^ (m & 7)) * 16);
+          uint4* p1 = reinterpret_cast<uint4*>(hbase + ((((2 * c + 1) & 7)) ^ (m & 7)) * 16);
+          uint4 w[2] = {*p0, *p1};
+          uint16_t* h = reinterpret_cast<uint16_t*>(w);
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            h[u] = Elem<E>::from_f32(
+                fmaf(P.scale, __uint_as_float(r[u]) * inv, Elem<E>::to_f32(h[u])));
+          *p0 = w[0];
+          *p1 = w[1];
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&accempty[a]);   // accumulator a may be overwritten
+      if (tiled && nn == kNT) {
+        // whole tile: two 2-D TMA stores once all four warps updated their rows
+        ptx::fence_proxy_async_smem();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (warp == 0) {
+          if (lane == 0) {
+            ptx::tma_store_2d(&P.tmY, (int)(ycol0 + n0), m0, ys);
+            ptx::tma_store_2d(&P.tmY, (int)(ycol0 + n0 + 64), m0, ys + L::kYHalf);
+            ptx::bulk_commit();
+            ptx::bulk_wait_read_all();                  // the stage may be refilled
+          }
+          __syncwarp();
+        }
+      } else {
+        // coalesced 16-byte stores of this warp's valid rows: lane -> (row pair, chunk)
+        for (int i = 0; i < 16; ++i) {
+          const int mr = warp * 32 + 2 * i + (lane >> 4);
+          const int q = lane & 15;
+          if (mr < valid && q * 8 < nn) {
+            const int tk = P.perm ? P.perm[m0 + mr] : m0 + mr;
+            const uint4 v = *reinterpret_cast<const uint4*>(
+                ys + (q >> 3) * L::kYHalf + mr * 128 + (((q & 7) ^ (mr & 7)) * 16));
+            *reinterpret_cast<uint4*>(ycol + (size_t)tk * P.ldy + n0 + q * 8) = v;
+          }
+        }
+        ptx::fence_proxy_async_smem();   // generic accesses before the next async refill
+        __syncwarp();
+      }
+      if (lane == 0) ptx::mbar_arrive(&empty[s]);
+    }
+    if (warp == 0 && lane == 0) ptx::bulk_wait_all();
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 0) ptx::tmem_dealloc(tmem, kNT);
-  if (!ok && tid == 0) atomicAdd(P.bad_meta, 1);
+  if (warp == 8) ptx::tmem_dealloc(tmem, 2 * kNT);
+  if (!ok && lane == 0) atomicAdd(P.bad_meta, 1);
 }
 
 template <typename E, int R>
@@ -536,7 +671,7 @@ cudaError_t shrink_tc_launch(const ShrinkArgs& a, const SegArgs& sg, lora_dtype 
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(max_tiles * KS, a.n_slices, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(kShrThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -563,6 +698,14 @@ cudaError_t expand_tc_launch(const ExpandArgs& a, const SegArgs& sg, lora_dtype 
     P.D_out[i] = a.D_out[i];
     max_nt = max(max_nt, (a.D_out[i] + kNT - 1) / kNT);
   }
+  {
+    cudaError_t e = encode_tmap_2d(&P.tmY, dt, a.y, (uint64_t)a.ldy, (uint64_t)a.T,
+                                   (uint64_t)a.ldy * 2, 64, kTM, 128);
+    if (e == cudaSuccess)
+      e = encode_tmap_2d(&P.tmYg, dt, a.y, (uint64_t)a.ldy, (uint64_t)a.T, (uint64_t)a.ldy * 2,
+                         64, 1, 128);
+    if (e != cudaSuccess) return e;
+  }
   const MetaHeader* hdr = reinterpret_cast<const MetaHeader*>(a.meta);
   P.buf = a.buf;
   P.buf_slice_stride = a.buf_slice_stride;
@@ -580,12 +723,18 @@ cudaError_t expand_tc_launch(const ExpandArgs& a, const SegArgs& sg, lora_dtype 
   P.bad_index = const_cast<int*>(&hdr->bad_index);
   P.bad_meta = const_cast<int*>(&hdr->bad_meta);
   const int max_tiles = (a.T + kTM - 1) / kTM + sg.n_seg;
+  // n-tiles per CTA: about three waves of one CTA per SM over all the work
+  const long units = (long)max_tiles * max_nt * a.n_slices;
+  int NJ = (int)((units + 3 * 148 - 1) / (3 * 148));
+  NJ = NJ < 1 ? 1 : (NJ > max_nt ? max_nt : NJ);
+  P.NJ = NJ;
+  P.n_chunks = (max_nt + NJ - 1) / NJ;
   auto kern = sgmv_expand_tc_kernel<E, R>;
   const size_t smem = ExpandSmem<R>::kTotal;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(max_tiles, max_nt, a.n_slices), kThreads, smem, st>>>(P);
+  kern<<<dim3(max_tiles * P.n_chunks, a.n_slices, 1), kExpThreads, smem, st>>>(P);
   return cudaGetLastError();
 }
 
