@@ -54,6 +54,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// The same bounded wait for kernels with many waits in a row: it gives up at
+// once when another thread of the CTA has already timed out (*abort != 0), and
+// sets *abort itself on a timeout, so a broken pipeline ends after one
+// timeout instead of one per wait.
+__device__ __forceinline__ bool mbar_wait_ff(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const uint32_t addr = smem_u32(bar);
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((it & 63) == 0) {
+      if (*abort) return false;
+      if (it == 0) {
+        t0 = globaltimer_ns();
+      } else if (globaltimer_ns() - t0 > 1000000000ull) {
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- bulk copies
 // 1-D bulk copy global -> shared (16-byte aligned addresses, size % 16 == 0),
 // completion counted on an mbarrier in bytes.

@@ -113,10 +113,10 @@ __device__ void validate_segments(const int32_t* ss, const int32_t* sa, int n_se
 // The per-token grouping in the workspace was built for (T, S): otherwise its
 // positions are not known to lie in this call's buffers, so nothing is done
 // and the error is counted once (the error counters head the workspace).
-__device__ bool grouped_meta_ok(int* counters, int T, int S) {
+__device__ bool grouped_meta_ok(int* counters, int T, int S, bool count) {
   const MetaHeader* h = reinterpret_cast<const MetaHeader*>(counters);
   if (h->T == T && h->S == S) return true;
-  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0)
+  if (count && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
     atomicAdd(&reinterpret_cast<MetaHeader*>(counters)->bad_meta, 1);
   return false;
 }
@@ -184,7 +184,7 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   if (blockIdx.x == 0 && slice == 0 && !P.implicit_slots)
     validate_segments(P.seg_starts, P.seg_adapter, P.n_seg, P.T, P.S, P.bad_index, P.bad_meta);
   // grouping metadata must have been built for this call's sizes
-  const bool meta_ok = !P.implicit_slots || grouped_meta_ok(P.bad_index, P.T, P.S);
+  const bool meta_ok = !P.implicit_slots || grouped_meta_ok(P.bad_index, P.T, P.S, tid == 0);
   if (warp == 0) {
     TileInfo ti;
     const bool found = meta_ok && find_tile(blockIdx.x / KS, P.seg_starts, P.seg_adapter,
@@ -335,6 +335,30 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   if (!ok && tid == 0) atomicAdd(P.bad_meta, 1);
 }
 
+// ---------------------------------------------------------------- expand
+// Persistent: one CTA per SM walks a contiguous range of (slice, tile, n-tile)
+// pairs.  The pairs are ordered slice-major, then by tile, then by 128-column
+// output tile, and weighted by the bytes they move (B tile + y rows read and
+// written + a fixed cost), so every CTA gets the same share of the traffic
+// whatever the mix of full and nearly empty tiles.  A CTA lists its tile runs
+// (a tile and the n-tiles of it that fall in its range) once, then runs one
+// continuous pipeline over them:
+//   load warps   B tile + y tile of each pair into a ring of stages; the
+//                hi / lo operand of each run (double-buffered)
+//   MMA warp     acc = hi . B^T + lo . B^T into one of two TMEM accumulators;
+//                a tile of <= 64 rows swaps the operands (M = 128 output
+//                columns, N = its rows rounded to 16) so the epilogue only
+//                touches the rows that exist
+//   epilogue     y += scale * acc, one rounding; two warps per TMEM lane
+//                quadrant split the columns (or the token chunks)
+struct ExpRun {
+  int m0, valid, adapter, slice, j0, j1;
+};
+constexpr int kMaxRuns = 64;
+constexpr int kMaxSegTC = 2048;          // longer segment lists use the item kernels
+constexpr int kMaxSegChunks = kMaxSegTC / 32 + 1;
+constexpr int kSwapMax = 64;             // tiles of at most this many rows swap operands
+
 struct ExpandTCParams {
   CUtensorMap tmB[LORA_MAX_SLICES];      // B_i as [S*D_out_i rows, r cols], box {r, 128}
   CUtensorMap tmY;                       // y as [T rows, ldy cols], box {64, 128}, 128B swizzle
@@ -351,7 +375,6 @@ struct ExpandTCParams {
   const int32_t* perm;                   // row p of a tile is token perm[p]; null = identity
   int implicit_slots;                    // > 0: segment g is slot g (per-token grouping)
   int T, S, n_slices;
-  int NJ, n_chunks;                      // each CTA walks NJ consecutive 128-column tiles
   float scale;
   int* bad_index;
   int* bad_meta;
@@ -359,23 +382,166 @@ struct ExpandTCParams {
 
 template <int R>
 struct ExpandSmem {
-  static constexpr int kYS = 3;                           // {B tile, y tile} ring stages
   static constexpr int kRowBytes = R * 2;                 // = swizzle width of the operands
   static constexpr int kBBytes = kNT * kRowBytes;
   static constexpr int kHBytes = kTM * kRowBytes;
   static constexpr int kYHalf = kTM * 128;                // 64 columns x 128 rows, 128B swizzle
   static constexpr int kYBytes = 2 * kYHalf;
-  static constexpr size_t kOffB = 0;
-  static constexpr size_t kOffHi = kOffB + (size_t)kYS * kBBytes;
-  static constexpr size_t kOffLo = kOffHi + kHBytes;
-  static constexpr size_t kOffY = kOffLo + kHBytes;
-  static constexpr size_t kOffBar = kOffY + (size_t)kYS * kYBytes;
-  static constexpr size_t kTotal = kOffBar + 8 * (2 * kYS + 5) + 64 + 1024;
+  static constexpr int kYS = R == 64 ? 3 : (R == 32 ? 4 : 5);   // {B tile, y tile} stages
+  static constexpr size_t kOffY = 0;
+  static constexpr size_t kOffB = kOffY + (size_t)kYS * kYBytes;
+  static constexpr size_t kOffHL = kOffB + (size_t)kYS * kBBytes;     // [2] x {hi, lo}
+  static constexpr size_t kOffInv = kOffHL + 4 * (size_t)kHBytes;     // float [2][128]
+  static constexpr size_t kOffTok = kOffInv + 2 * kTM * 4;            // int [2][128]
+  static constexpr size_t kOffRun = kOffTok + 2 * kTM * 4;            // ExpRun [kMaxRuns]
+  static constexpr size_t kOffChunk = kOffRun + kMaxRuns * sizeof(ExpRun);   // int64 [chunks]
+  static constexpr size_t kOffBar = kOffChunk + 8 * kMaxSegChunks;
+  static constexpr int kNBar = 2 * kYS + 8;
+  static constexpr size_t kOffMisc = kOffBar + 8 * kNBar;             // tmem, n_runs, next
+  static constexpr size_t kTotal = kOffMisc + 64 + 1024;
 };
 
-// warps 0-3: epilogue (TMEM lane quadrant = warp), warps 4-7: loads (one per
-// SM sub-partition, so small copies issue four-wide), warp 8: MMA issue.
-constexpr int kExpThreads = 288;
+// Bytes a pair moves, in units the schedule balances: the B tile, the valid
+// y rows read and written, and a fixed per-pair cost.
+template <int R>
+__device__ __forceinline__ int64_t pair_weight(int valid) {
+  return (int64_t)kNT * R * 2 + 512 * (int64_t)valid + 4096;
+}
+
+struct SegView {
+  const int32_t* ss;
+  const int32_t* sa;
+  int n_seg, T, S, implicit_slots;
+  // segment s clamped into [0, T]; adapter -1 when it has none or is out of range
+  __device__ __forceinline__ void get(int s, int& a, int& b, int& ad) const {
+    a = 0; b = 0; ad = -1;
+    if (s < n_seg) {
+      a = min(max(ss[s], 0), T);
+      b = max(a, min(max(ss[s + 1], 0), T));
+      ad = implicit_slots ? (s < implicit_slots ? s : -1) : sa[s];
+      if (ad < 0 || ad >= S) ad = -1;
+    }
+  }
+};
+
+// Per n-tile weight of one segment: its full tiles and its partial last tile.
+template <int R>
+__device__ __forceinline__ int64_t seg_weight(int a, int b, int ad) {
+  if (ad < 0) return 0;
+  const int len = b - a;
+  const int rem = len % kTM;
+  return (int64_t)(len / kTM) * pair_weight<R>(kTM) + (rem ? pair_weight<R>(rem) : 0);
+}
+
+// Warp 0 of the CTA: per-chunk (32 segments) weights into chunkW, total
+// returned in every lane.
+template <int R>
+__device__ int64_t seg_chunk_weights(const SegView& sv, int64_t* chunkW) {
+  const int lane = threadIdx.x & 31;
+  const int nch = (sv.n_seg + 31) / 32;
+  int64_t total = 0;
+  for (int c0 = 0; c0 < nch; c0 += 4) {
+    int64_t w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {          // all loads first, then the reductions
+      int a, b, ad;
+      sv.get((c0 + u) * 32 + lane, a, b, ad);
+      w[u] = seg_weight<R>(a, b, ad);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      int64_t v = w[u];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0 && c0 + u < nch) chunkW[c0 + u] = v;
+      total += c0 + u < nch ? v : 0;
+    }
+  }
+  return total;
+}
+
+__device__ __forceinline__ int64_t ceil_pos(int64_t num, int64_t w) {
+  return num <= 0 ? 0 : (num + w - 1) / w;
+}
+
+// Warp-cooperative: the tile runs whose pair start positions fall in
+// [lo, hi), in schedule order, at most kMaxRuns of them.  Returns the count;
+// *next is hi when the list is complete, else where the next list starts.
+template <int R>
+__device__ int build_runs(const SegView& sv, const int64_t* chunkW, int64_t Wt,
+                          const int* ntiles, int n_slices, int64_t lo, int64_t hi,
+                          ExpRun* runs, int64_t* next) {
+  const int lane = threadIdx.x & 31;
+  const int nch = (sv.n_seg + 31) / 32;
+  int n = 0;
+  int64_t pos = 0;
+  *next = hi;
+  for (int i = 0; i < n_slices && pos < hi; ++i) {
+    const int64_t nt = ntiles[i];
+    if (pos + nt * Wt <= lo) {
+      pos += nt * Wt;
+      continue;
+    }
+    int64_t cpos = pos;
+    for (int c = 0; c < nch && cpos < hi; ++c) {
+      const int64_t cw = nt * chunkW[c];
+      if (cpos + cw <= lo || cw == 0) {
+        cpos += cw;
+        continue;
+      }
+      int a, b, ad;
+      sv.get(c * 32 + lane, a, b, ad);
+      const int64_t sw = nt * seg_weight<R>(a, b, ad);
+      int64_t incl = sw;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int64_t spos = cpos + incl - sw;
+      unsigned mask = __ballot_sync(0xffffffffu, sw > 0 && spos < hi && spos + sw > lo);
+      while (mask) {
+        const int l = __ffs(mask) - 1;
+        mask &= mask - 1;
+        const int a_l = __shfl_sync(0xffffffffu, a, l);
+        const int len = __shfl_sync(0xffffffffu, b, l) - a_l;
+        const int ad_l = __shfl_sync(0xffffffffu, ad, l);
+        const int64_t sp = __shfl_sync(0xffffffffu, spos, l);
+        const int ntk = (len + kTM - 1) / kTM;
+        for (int k0 = 0; k0 < ntk; k0 += 32) {
+          const int k = k0 + lane;
+          const int valid = k < ntk ? min(kTM, len - k * kTM) : 0;
+          const int64_t w = pair_weight<R>(valid);
+          const int64_t tpos = sp + nt * (int64_t)k * pair_weight<R>(kTM);
+          const int jl = (int)(ceil_pos(lo - tpos, w) < nt ? ceil_pos(lo - tpos, w) : nt);
+          const int jh = (int)(ceil_pos(hi - tpos, w) < nt ? ceil_pos(hi - tpos, w) : nt);
+          const bool has = k < ntk && jl < jh;
+          const unsigned hm = __ballot_sync(0xffffffffu, has);
+          const int rank = __popc(hm & ((1u << lane) - 1));
+          if (has && n + rank < kMaxRuns)
+            runs[n + rank] = ExpRun{a_l + k * kTM, valid, ad_l, i, jl, jh};
+          const int cnt = __popc(hm);
+          if (n + cnt > kMaxRuns) {
+            // the first run that did not fit starts the next list
+            const int64_t resume = max(lo, tpos);
+            const unsigned over = __ballot_sync(0xffffffffu, has && n + rank == kMaxRuns);
+            *next = __shfl_sync(0xffffffffu, resume, __ffs(over) - 1);
+            return kMaxRuns;
+          }
+          n += cnt;
+        }
+      }
+      cpos += cw;
+    }
+    pos += nt * Wt;
+  }
+  return n;
+}
+
+// warps 0-7: epilogue (TMEM lane quadrant = warp % 4, column half = warp / 4),
+// warps 8-11: loads (one per SM sub-partition), warp 12: MMA issue.
+constexpr int kExpThreads = 416;
+constexpr int kExpLoad0 = 8, kExpMma = 12;
 
 template <typename E, int R>
 __global__ void __launch_bounds__(kExpThreads, 1)
@@ -383,258 +549,376 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   using L = ExpandSmem<R>;
   constexpr int kYS = L::kYS;
   constexpr bool kBF = std::is_same<E, __nv_bfloat16>::value;
-  constexpr uint32_t kIdesc = ptx::umma_idesc_f16(kBF, kTM, kNT);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int slice = blockIdx.y;
-  const int Dout = P.D_out[slice];
-  const int ntiles = (Dout + kNT - 1) / kNT;
-  const int chunk = blockIdx.x % P.n_chunks;
-  const int j0 = chunk * P.NJ, j1 = min(ntiles, j0 + P.NJ);
-  if (j0 >= j1) return;
-  const int nj = j1 - j0;
 
   extern __shared__ char smem_raw[];
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                        ~uintptr_t(1023));
-  char* sB = smem + L::kOffB;
-  char* sHi = smem + L::kOffHi;
-  char* sLo = smem + L::kOffLo;
   char* sY = smem + L::kOffY;
+  char* sB = smem + L::kOffB;
+  char* sHL = smem + L::kOffHL;
+  float* sInv = reinterpret_cast<float*>(smem + L::kOffInv);
+  int* sTok = reinterpret_cast<int*>(smem + L::kOffTok);
+  ExpRun* runs = reinterpret_cast<ExpRun*>(smem + L::kOffRun);
+  int64_t* chunkW = reinterpret_cast<int64_t*>(smem + L::kOffChunk);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* empty = full + kYS;
   uint64_t* accfull = empty + kYS;       // [2]
   uint64_t* accempty = accfull + 2;      // [2]
-  uint64_t* hilo = accempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(hilo + 1);
-  int* sinfo = reinterpret_cast<int*>(tmem_slot + 4);
+  uint64_t* hlfull = accempty + 2;       // [2]
+  uint64_t* hlempty = hlfull + 2;        // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
+  int* sNRuns = reinterpret_cast<int*>(tmem_slot + 1);
+  int64_t* sRange = reinterpret_cast<int64_t*>(smem + L::kOffMisc + 8);   // lo, hi, Wt, next
+  volatile int* sAbort = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 48);
 
-  if (blockIdx.x == 0 && slice == 0 && !P.implicit_slots)
+  const SegView sv{P.seg_starts, P.seg_adapter, P.n_seg, P.T, P.S, P.implicit_slots};
+  if (blockIdx.x == 0 && !P.implicit_slots)
     validate_segments(P.seg_starts, P.seg_adapter, P.n_seg, P.T, P.S, P.bad_index, P.bad_meta);
-  const bool meta_ok = !P.implicit_slots || grouped_meta_ok(P.bad_index, P.T, P.S);
-  if (warp == 0) {
-    TileInfo ti;
-    const bool found = meta_ok && find_tile(blockIdx.x / P.n_chunks, P.seg_starts, P.seg_adapter,
-                                            P.n_seg, P.T, ti, P.implicit_slots);
-    if (lane == 0) {
-      sinfo[0] = found && ti.adapter >= 0 && ti.adapter < P.S ? 1 : 0;
-      sinfo[1] = ti.m0;
-      sinfo[2] = ti.valid;
-      sinfo[3] = ti.adapter;
-    }
+  int ntiles[LORA_MAX_SLICES];
+  int64_t sum_nt = 0;
+  for (int i = 0; i < P.n_slices; ++i) {
+    ntiles[i] = (P.D_out[i] + kNT - 1) / kNT;
+    sum_nt += ntiles[i];
   }
-  __syncthreads();
-  if (!sinfo[0]) return;                 // no tile, or rows without an adapter: untouched
-  const int m0 = sinfo[1], valid = sinfo[2], adapter = sinfo[3];
-  const int64_t ycol0 = P.y_col_off[slice];
-  E* ycol = static_cast<E*>(P.y) + ycol0;
-  // whole 128-row tile of consecutive tokens: y moves as 2-D TMA tiles
-  const bool tiled = P.perm == nullptr && valid == kTM;
 
+  if (warp == kExpMma) {
+    // this CTA's share of the weighted pair sequence
+    const bool meta_ok = !P.implicit_slots || grouped_meta_ok(P.bad_index, P.T, P.S, lane == 0);
+    const int64_t Wt = meta_ok ? seg_chunk_weights<R>(sv, chunkW) : 0;
+    const int64_t W = Wt * sum_nt;
+    if (lane == 0) {
+      sRange[0] = W * (int64_t)blockIdx.x / gridDim.x;
+      sRange[1] = W * (int64_t)(blockIdx.x + 1) / gridDim.x;
+      sRange[2] = Wt;
+    }
+    __syncwarp();
+    ptx::tmem_alloc(tmem_slot, 2 * kNT);
+    ptx::tmem_relinquish();
+  }
   if (tid == 0) {
+    *sAbort = 0;
     for (int s = 0; s < kYS; ++s) {
       ptx::mbar_init(&full[s], 4);       // one arrival per load warp
-      ptx::mbar_init(&empty[s], 4);      // one arrival per epilogue warp
+      ptx::mbar_init(&empty[s], 8);      // one arrival per epilogue warp
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&accfull[a], 1);
-      ptx::mbar_init(&accempty[a], 4);
+      ptx::mbar_init(&accempty[a], 8);
+      ptx::mbar_init(&hlfull[a], 4);
+      ptx::mbar_init(&hlempty[a], 8);
     }
-    ptx::mbar_init(hilo, 4);
     ptx::fence_mbar_init();
-    ptx::prefetch_tensormap(&P.tmB[slice]);
-    ptx::prefetch_tensormap(tiled ? &P.tmY : &P.tmYg);
-  }
-  if (warp == 8) {
-    ptx::tmem_alloc(tmem_slot, 2 * kNT);
-    ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  int64_t lo = sRange[0];
+  const int64_t hi = sRange[1], Wt = sRange[2];
   bool ok = true;
+  // pipeline positions, continued across run lists: pair p, run u
+  int p = 0, u = 0;
+  // epilogue: a TMA store of half h whose stage is released once it was read
+  int deferred = -1;
 
-  if (warp >= 4 && warp < 8) {
-    // ---- loads: B tile and y tile of n-tile j into stage j % kYS
-    const int pw = warp - 4;
-    const int ngroups = (valid + 3) / 4;
-    for (int j = 0; j < nj; ++j) {
-      const int s = j % kYS;
-      if (j >= kYS) ok &= ptx::mbar_wait(&empty[s], ((j / kYS) - 1) & 1);
-      const int n0 = (j0 + j) * kNT;
-      char* ys = sY + (size_t)s * L::kYBytes;
-      // ops of this n-tile: 2 y halves x ngroups 4-row gathers, dealt out over
-      // the four load warps (op o -> warp o % 4, lane o / 4)
-      int my_ops = 0;
-      if (!tiled)
-        for (int o = pw; o < 2 * ngroups; o += 4) ++my_ops;
-      const uint32_t bytes = (uint32_t)(my_ops * 512) +
-                             (pw == 0 ? (uint32_t)L::kBBytes + (tiled ? (uint32_t)L::kYBytes : 0u) : 0u);
+  while (lo < hi) {
+    if (warp == kExpMma) {
+      int64_t nx;
+      const int n = build_runs<R>(sv, chunkW, Wt, ntiles, P.n_slices, lo, hi, runs, &nx);
       if (lane == 0) {
-        ptx::mbar_arrive_expect_tx(&full[s], bytes);
-        if (pw == 0) {
-          ptx::tma_load_2d(sB + (size_t)s * L::kBBytes, &P.tmB[slice], 0, adapter * Dout + n0,
-                           &full[s]);
-          if (tiled) {
-            ptx::tma_load_2d(ys, &P.tmY, (int)(ycol0 + n0), m0, &full[s]);
-            ptx::tma_load_2d(ys + L::kYHalf, &P.tmY, (int)(ycol0 + n0 + 64), m0, &full[s]);
-          }
-        }
-      }
-      __syncwarp();
-      if (!tiled) {
-        for (int o = pw + 4 * lane; o < 2 * ngroups; o += 128) {
-          const int g = o >> 1, h = o & 1;
-          int rr[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int mm = 4 * g + q < valid ? 4 * g + q : 0;
-            rr[q] = P.perm ? P.perm[m0 + mm] : m0 + mm;
-          }
-          ptx::tma_gather4(ys + h * L::kYHalf + g * 512, &P.tmYg, (int)(ycol0 + n0 + 64 * h),
-                           rr[0], rr[1], rr[2], rr[3], &full[s]);
-        }
+        *sNRuns = n;
+        sRange[3] = nx;
       }
     }
-  } else if (warp == 8) {
-    // ---- MMA issue: acc[j & 1] = hi . B^T + lo . B^T
-    if (lane == 0) {
-      ok &= ptx::mbar_wait(hilo, 0);
-      const uint32_t hb = ptx::smem_u32(sHi), lb = ptx::smem_u32(sLo);
-      for (int j = 0; j < nj; ++j) {
-        const int s = j % kYS, a = j & 1;
-        ok &= ptx::mbar_wait(&full[s], (j / kYS) & 1);
-        if (j >= 2) ok &= ptx::mbar_wait(&accempty[a], ((j / 2) - 1) & 1);
-        ptx::tc_fence_after();
-        const uint32_t bb = ptx::smem_u32(sB + (size_t)s * L::kBBytes);
-        const uint32_t acc = tmem + a * kNT;
-#pragma unroll
-        for (int ks = 0; ks < R / 16; ++ks)
-          ptx::tc_mma_f16(acc, ptx::umma_desc_kmajor(hb + ks * 32, L::kRowBytes),
-                          ptx::umma_desc_kmajor(bb + ks * 32, L::kRowBytes), kIdesc,
-                          ks > 0 ? 1u : 0u);
-#pragma unroll
-        for (int ks = 0; ks < R / 16; ++ks)
-          ptx::tc_mma_f16(acc, ptx::umma_desc_kmajor(lb + ks * 32, L::kRowBytes),
-                          ptx::umma_desc_kmajor(bb + ks * 32, L::kRowBytes), kIdesc, 1u);
-        ptx::tc_commit(&accfull[a]);
-      }
-    }
-  } else {
-    // ---- epilogue warps 0-3: row m = TMEM lane 32 * warp + lane
-    const int m = warp * 32 + lane;
-    const int tok = m < valid ? (P.perm ? P.perm[m0 + m] : m0 + m) : 0;
-    // row m's intermediate -> hi / lo operand rows (swizzled K-major), after an
-    // exact power-of-two rescale 2^(7-e), e the exponent of max |buf| of the row
-    float inv = 1.f;
-    {
-      const float4* brow = reinterpret_cast<const float4*>(
-          P.buf + (size_t)slice * P.buf_slice_stride + (size_t)tok * R);
-      float mx = 0.f;
-#pragma unroll
-      for (int q = 0; q < R / 4; ++q) {
-        const float4 f = m < valid ? brow[q] : make_float4(0.f, 0.f, 0.f, 0.f);
-        mx = fmaxf(fmaxf(fmaxf(mx, fabsf(f.x)), fmaxf(fabsf(f.y), fabsf(f.z))), fabsf(f.w));
-      }
-      int e = ((__float_as_int(mx) >> 23) & 0xff) - 127;
-      e = (mx > 0.f && e > -100 && e < 100) ? e : 0;
-      const float sc = __int_as_float((127 - e + 7) << 23);
-      inv = __int_as_float((127 + e - 7) << 23);
-#pragma unroll
-      for (int c = 0; c < R / 8; ++c) {
-        float4 f0 = make_float4(0.f, 0.f, 0.f, 0.f), f1 = f0;
-        if (m < valid) {
-          f0 = brow[2 * c];
-          f1 = brow[2 * c + 1];
-        }
-        const float x8[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-        uint16_t hi[8], lo[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float xv = x8[u] * sc;
-          hi[u] = Elem<E>::from_f32(xv);
-          lo[u] = Elem<E>::from_f32(xv - Elem<E>::to_f32(hi[u]));
-        }
-        const int off = m * L::kRowBytes + swz<L::kRowBytes>(m, c) * 16;
-        *reinterpret_cast<uint4*>(sHi + off) = *reinterpret_cast<const uint4*>(hi);
-        *reinterpret_cast<uint4*>(sLo + off) = *reinterpret_cast<const uint4*>(lo);
-      }
-    }
-    ptx::fence_proxy_async_smem();       // generic writes -> tensor-core operand reads
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(hilo);
+    __syncthreads();
+    const int n_runs = *sNRuns;
+    const int64_t next_lo = sRange[3];
 
-    for (int j = 0; j < nj; ++j) {
-      const int s = j % kYS, a = j & 1;
-      const int n0 = (j0 + j) * kNT, nn = min(kNT, Dout - n0);
-      ok &= ptx::mbar_wait(&accfull[a], (j / 2) & 1);
-      ok &= ptx::mbar_wait(&full[s], (j / kYS) & 1);
-      ptx::tc_fence_after();
-      char* ys = sY + (size_t)s * L::kYBytes;
-      // y tile layout: two 64-column halves, 128-byte rows, 16-byte chunk q of
-      // a row at position q ^ (row & 7)
-      for (int c = 0; c < kNT / 16; ++c) {
-        uint32_t r[16];
-        ptx::tc_ld16(tmem + a * kNT + ((uint32_t)(warp * 32) << 16) + c * 16, r);
-        ptx::tc_wait_ld();
-        if (m < valid) {
-          char* hbase = ys + (c >> 2) * L::kYHalf + m * 128;
-          uint4* p0 = reinterpret_cast<uint4*>(hbase + ((((2 * c) & 7)) ^ (m & 7)) * 16);
-          uint4* p1 = reinterpret_cast<uint4*>(hbase + ((((2 * c + 1) & 7)) ^ (m & 7)) * 16);
-          uint4 w[2] = {*p0, *p1};
-          uint16_t* h = reinterpret_cast<uint16_t*>(w);
+    if (warp >= kExpLoad0 && warp < kExpMma) {
+      // ---------------- loads
+      const int pw = warp - kExpLoad0;
+      const int lt = pw * 32 + lane;                 // operand row of this thread
+      int pl = p, ul = u;
+      for (int ri = 0; ri < n_runs; ++ri, ++ul) {
+        const ExpRun rn = runs[ri];
+        const int hb = ul & 1;
+        if (ul >= 2) ok &= ptx::mbar_wait_ff(&hlempty[hb], ((ul >> 1) - 1) & 1, sAbort);
+        // operand rows: token, hi / lo after an exact power-of-two rescale
+        // 2^(7-e) (e = exponent of the row's max |buf|), and the inverse scale
+        {
+          const int m = lt;
+          const int tok = m < rn.valid ? (P.perm ? P.perm[rn.m0 + m] : rn.m0 + m) : -1;
+          const float4* brow = reinterpret_cast<const float4*>(
+              P.buf + (size_t)rn.slice * P.buf_slice_stride + (size_t)(tok < 0 ? 0 : tok) * R);
+          float4 f[R / 4];
+          float mx = 0.f;
 #pragma unroll
-          for (int u = 0; u < 16; ++u)
-            h[u] = Elem<E>::from_f32(
-                fmaf(P.scale, __uint_as_float(r[u]) * inv, Elem<E>::to_f32(h[u])));
-          *p0 = w[0];
-          *p1 = w[1];
+          for (int q = 0; q < R / 4; ++q) {
+            f[q] = tok >= 0 ? brow[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+            mx = fmaxf(fmaxf(fmaxf(mx, fabsf(f[q].x)), fmaxf(fabsf(f[q].y), fabsf(f[q].z))),
+                       fabsf(f[q].w));
+          }
+          int e = ((__float_as_int(mx) >> 23) & 0xff) - 127;
+          e = (mx > 0.f && e > -100 && e < 100) ? e : 0;
+          const float sc = __int_as_float((127 - e + 7) << 23);
+          char* hiP = sHL + (size_t)(2 * hb) * L::kHBytes;
+          char* loP = hiP + L::kHBytes;
+#pragma unroll
+          for (int c = 0; c < R / 8; ++c) {
+            const float x8[8] = {f[2 * c].x, f[2 * c].y, f[2 * c].z, f[2 * c].w,
+                                 f[2 * c + 1].x, f[2 * c + 1].y, f[2 * c + 1].z, f[2 * c + 1].w};
+            uint16_t h8[8], l8[8];
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const float xv = x8[v] * sc;
+              h8[v] = Elem<E>::from_f32(xv);
+              l8[v] = Elem<E>::from_f32(xv - Elem<E>::to_f32(h8[v]));
+            }
+            const int off = m * L::kRowBytes + swz<L::kRowBytes>(m, c) * 16;
+            *reinterpret_cast<uint4*>(hiP + off) = *reinterpret_cast<const uint4*>(h8);
+            *reinterpret_cast<uint4*>(loP + off) = *reinterpret_cast<const uint4*>(l8);
+          }
+          sInv[hb * kTM + m] = __int_as_float((127 + e - 7) << 23);
+          sTok[hb * kTM + m] = tok;
+          ptx::fence_proxy_async_smem();   // generic writes -> tensor-core operand reads
         }
-      }
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&accempty[a]);   // accumulator a may be overwritten
-      if (tiled && nn == kNT) {
-        // whole tile: two 2-D TMA stores once all four warps updated their rows
-        ptx::fence_proxy_async_smem();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (warp == 0) {
+        asm volatile("bar.sync 4, 128;" ::: "memory");   // every row's token is known
+        if (lane == 0) ptx::mbar_arrive(&hlfull[hb]);
+        const int* toks = sTok + hb * kTM;
+        const int Dout = P.D_out[rn.slice];
+        const int64_t ycol0 = P.y_col_off[rn.slice];
+        const bool tiled = P.perm == nullptr && rn.valid == kTM;
+        const int ngroups = (rn.valid + 3) / 4;
+        int my_ops = 0;
+        if (!tiled)
+          for (int o = pw; o < 2 * ngroups; o += 4) ++my_ops;
+        for (int j = rn.j0; j < rn.j1; ++j, ++pl) {
+          const int s = pl % kYS;
+          if (pl >= kYS) ok &= ptx::mbar_wait_ff(&empty[s], ((pl / kYS) - 1) & 1, sAbort);
+          const int n0 = j * kNT;
+          char* ys = sY + (size_t)s * L::kYBytes;
+          const uint32_t bytes =
+              (uint32_t)(my_ops * 512) +
+              (pw == 0 ? (uint32_t)L::kBBytes + (tiled ? (uint32_t)L::kYBytes : 0u) : 0u);
           if (lane == 0) {
-            ptx::tma_store_2d(&P.tmY, (int)(ycol0 + n0), m0, ys);
-            ptx::tma_store_2d(&P.tmY, (int)(ycol0 + n0 + 64), m0, ys + L::kYHalf);
-            ptx::bulk_commit();
-            ptx::bulk_wait_read_all();                  // the stage may be refilled
+            ptx::mbar_arrive_expect_tx(&full[s], bytes);
+            if (pw == 0) {
+              ptx::tma_load_2d(sB + (size_t)s * L::kBBytes, &P.tmB[rn.slice], 0,
+                               rn.adapter * Dout + n0, &full[s]);
+              if (tiled) {
+                ptx::tma_load_2d(ys, &P.tmY, (int)(ycol0 + n0), rn.m0, &full[s]);
+                ptx::tma_load_2d(ys + L::kYHalf, &P.tmY, (int)(ycol0 + n0 + 64), rn.m0, &full[s]);
+              }
+            }
           }
           __syncwarp();
-        }
-      } else {
-        // coalesced 16-byte stores of this warp's valid rows: lane -> (row pair, chunk)
-        for (int i = 0; i < 16; ++i) {
-          const int mr = warp * 32 + 2 * i + (lane >> 4);
-          const int q = lane & 15;
-          if (mr < valid && q * 8 < nn) {
-            const int tk = P.perm ? P.perm[m0 + mr] : m0 + mr;
-            const uint4 v = *reinterpret_cast<const uint4*>(
-                ys + (q >> 3) * L::kYHalf + mr * 128 + (((q & 7) ^ (mr & 7)) * 16));
-            *reinterpret_cast<uint4*>(ycol + (size_t)tk * P.ldy + n0 + q * 8) = v;
+          if (!tiled) {
+            // 2 halves x ngroups 4-row gathers: op o -> warp o % 4, lane o / 4
+            for (int o = pw + 4 * lane; o < 2 * ngroups; o += 128) {
+              const int g = o >> 1, h = o & 1;
+              int rr[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) rr[q] = toks[4 * g + q < rn.valid ? 4 * g + q : 4 * g];
+              ptx::tma_gather4(ys + h * L::kYHalf + g * 512, &P.tmYg, (int)(ycol0 + n0 + 64 * h),
+                               rr[0], rr[1], rr[2], rr[3], &full[s]);
+            }
           }
         }
-        ptx::fence_proxy_async_smem();   // generic accesses before the next async refill
-        __syncwarp();
       }
-      if (lane == 0) ptx::mbar_arrive(&empty[s]);
+    } else if (warp == kExpMma) {
+      // ---------------- MMA issue
+      if (lane == 0) {
+        int pl = p, ul = u;
+        for (int ri = 0; ri < n_runs; ++ri, ++ul) {
+          const ExpRun rn = runs[ri];
+          const int hb = ul & 1;
+          const bool swap = rn.valid <= kSwapMax;
+          const uint32_t idesc =
+              ptx::umma_idesc_f16(kBF, kTM, swap ? (rn.valid + 15) / 16 * 16 : kNT);
+          ok &= ptx::mbar_wait_ff(&hlfull[hb], (ul >> 1) & 1, sAbort);
+          const uint32_t hiA = ptx::smem_u32(sHL + (size_t)(2 * hb) * L::kHBytes);
+          const uint32_t loA = hiA + L::kHBytes;
+          for (int j = rn.j0; j < rn.j1; ++j, ++pl) {
+            const int s = pl % kYS, a = pl & 1;
+            ok &= ptx::mbar_wait_ff(&full[s], (pl / kYS) & 1, sAbort);
+            if (pl >= 2) ok &= ptx::mbar_wait_ff(&accempty[a], ((pl >> 1) - 1) & 1, sAbort);
+            ptx::tc_fence_after();
+            const uint32_t bb = ptx::smem_u32(sB + (size_t)s * L::kBBytes);
+            const uint32_t acc = tmem + a * kNT;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              const uint32_t op = half ? loA : hiA;
+#pragma unroll
+              for (int ks = 0; ks < R / 16; ++ks) {
+                const uint64_t dOp = ptx::umma_desc_kmajor(op + ks * 32, L::kRowBytes);
+                const uint64_t dB = ptx::umma_desc_kmajor(bb + ks * 32, L::kRowBytes);
+                ptx::tc_mma_f16(acc, swap ? dB : dOp, swap ? dOp : dB, idesc,
+                                (half | ks) ? 1u : 0u);
+              }
+            }
+            ptx::tc_commit(&accfull[a]);
+          }
+        }
+      }
+      __syncwarp();
+    } else {
+      // ---------------- epilogue warps 0-7
+      const int q = warp & 3, h = warp >> 2;
+      int pl = p, ul = u;
+      for (int ri = 0; ri < n_runs; ++ri, ++ul) {
+        const ExpRun rn = runs[ri];
+        const int hb = ul & 1;
+        const bool swap = rn.valid <= kSwapMax;
+        ok &= ptx::mbar_wait_ff(&hlfull[hb], (ul >> 1) & 1, sAbort);
+        const int* toks = sTok + hb * kTM;
+        const float* invs = sInv + hb * kTM;
+        const int m = q * 32 + lane;                  // row of this thread (normal layout)
+        const int tok = toks[m];
+        const float inv = invs[m];
+        const int Dout = P.D_out[rn.slice];
+        E* ycol = static_cast<E*>(P.y) + P.y_col_off[rn.slice];
+        const int64_t ycol0 = P.y_col_off[rn.slice];
+        const bool tiled = P.perm == nullptr && rn.valid == kTM;
+        for (int j = rn.j0; j < rn.j1; ++j, ++pl) {
+          const int s = pl % kYS, a = pl & 1;
+          const int n0 = j * kNT, nn = min(kNT, Dout - n0);
+          ok &= ptx::mbar_wait_ff(&accfull[a], (pl >> 1) & 1, sAbort);
+          ok &= ptx::mbar_wait_ff(&full[s], (pl / kYS) & 1, sAbort);
+          ptx::tc_fence_after();
+          if (deferred >= 0) {
+            // the previous TMA store of this warp's half has been read: its stage is free
+            if (lane == 0) {
+              ptx::bulk_wait_read_all();
+              ptx::mbar_arrive(&empty[deferred]);
+            }
+            deferred = -1;
+            __syncwarp();
+          }
+          char* ys = sY + (size_t)s * L::kYBytes;
+          const uint32_t tacc = tmem + a * kNT + ((uint32_t)(q * 32) << 16);
+          if (!swap) {
+            // thread = row m, columns 64h .. 64h+63 = y half h
+            if (q * 32 < rn.valid) {
+              uint32_t r[64];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) ptx::tc_ld16(tacc + 64 * h + 16 * k, r + 16 * k);
+              ptx::tc_wait_ld();
+              if (m < rn.valid) {
+                char* row = ys + h * L::kYHalf + m * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  uint4* pc = reinterpret_cast<uint4*>(row + ((c ^ (m & 7)) << 4));
+                  uint4 w = *pc;
+                  uint16_t* hw = reinterpret_cast<uint16_t*>(&w);
+#pragma unroll
+                  for (int v = 0; v < 8; ++v)
+                    hw[v] = Elem<E>::from_f32(fmaf(P.scale, __uint_as_float(r[8 * c + v]) * inv,
+                                                   Elem<E>::to_f32(hw[v])));
+                  *pc = w;
+                }
+              }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&accempty[a]);
+            if (tiled && nn == kNT) {
+              // whole tile: one 2-D TMA store per half once its four warps are done
+              ptx::fence_proxy_async_smem();
+              asm volatile("bar.sync %0, 128;" ::"r"(1 + h) : "memory");
+              if (q == 0) {
+                if (lane == 0) {
+                  ptx::tma_store_2d(&P.tmY, (int)(ycol0 + n0 + 64 * h), rn.m0,
+                                    ys + h * L::kYHalf);
+                  ptx::bulk_commit();
+                }
+                deferred = s;
+              }
+            } else {
+              // rows 32q .. 32q+31 of half h: lane -> (row 4i + lane / 8, chunk lane % 8)
+#pragma unroll 2
+              for (int i = 0; i < 8; ++i) {
+                const int lr = 4 * i + (lane >> 3), ch = lane & 7;
+                const int mr = q * 32 + lr;
+                const int tk = __shfl_sync(0xffffffffu, tok, lr);
+                if (mr < rn.valid && 64 * h + 8 * ch < nn) {
+                  const uint4 v = *reinterpret_cast<const uint4*>(
+                      ys + h * L::kYHalf + mr * 128 + ((ch ^ (mr & 7)) << 4));
+                  *reinterpret_cast<uint4*>(ycol + (size_t)tk * P.ldy + n0 + 64 * h + 8 * ch) = v;
+                }
+              }
+              ptx::fence_proxy_async_smem();
+            }
+          } else {
+            // swapped: thread = output column 32q + lane; token chunks of 16
+            // alternate between the two warps of the quadrant
+            const int col = q * 32 + lane;
+            const int hc = col >> 6, cc = col & 63;
+            char* cbase = ys + hc * L::kYHalf + (cc & 7) * 2;
+            const int nch = (rn.valid + 15) / 16;
+            for (int k = h; k < nch; k += 2) {
+              uint32_t r[16];
+              ptx::tc_ld16(tacc + 16 * k, r);
+              ptx::tc_wait_ld();
+#pragma unroll
+              for (int v = 0; v < 16; ++v) {
+                const int t = 16 * k + v;
+                if (t < rn.valid) {
+                  uint16_t* py = reinterpret_cast<uint16_t*>(cbase + t * 128 + (((cc >> 3) ^ (t & 7)) << 4));
+                  *py = Elem<E>::from_f32(
+                      fmaf(P.scale, __uint_as_float(r[v]) * invs[t], Elem<E>::to_f32(*py)));
+                }
+              }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&accempty[a]);
+            asm volatile("bar.sync 3, 256;" ::: "memory");   // every column of every row done
+            // rows 0 .. valid-1, 16 chunks each: e -> (row e / 16, chunk e % 16)
+            for (int e = warp * 32 + lane; e < rn.valid * 16; e += 256) {
+              const int mr = e >> 4, hh = (e >> 3) & 1, ch = e & 7;
+              if (64 * hh + 8 * ch < nn) {
+                const uint4 v = *reinterpret_cast<const uint4*>(
+                    ys + hh * L::kYHalf + mr * 128 + ((ch ^ (mr & 7)) << 4));
+                *reinterpret_cast<uint4*>(ycol + (size_t)toks[mr] * P.ldy + n0 + 64 * hh + 8 * ch) = v;
+              }
+            }
+            ptx::fence_proxy_async_smem();
+          }
+          __syncwarp();
+          if (lane == 0 && deferred != s) ptx::mbar_arrive(&empty[s]);
+        }
+        // done with this run's tokens and scales
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&hlempty[hb]);
+      }
     }
-    if (warp == 0 && lane == 0) ptx::bulk_wait_all();
+    // advance the pipeline positions past this list
+    for (int ri = 0; ri < n_runs; ++ri) p += runs[ri].j1 - runs[ri].j0;
+    u += n_runs;
+    __syncthreads();                               // the run list may be rebuilt
+    lo = next_lo;
   }
+  if (warp < kExpLoad0 && deferred >= 0 && lane == 0) ptx::bulk_wait_read_all();
+  if (warp < kExpLoad0 && lane == 0) ptx::bulk_wait_all();
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 8) ptx::tmem_dealloc(tmem, 2 * kNT);
-  if (!ok && lane == 0) atomicAdd(P.bad_meta, 1);
+  if (*sAbort) {
+    // a wait timed out: let copies still in flight land before the CTA's
+    // shared memory is released
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (ptx::globaltimer_ns() - t0 < 50000ull) {
+    }
+  }
+  if (warp == kExpMma) ptx::tmem_dealloc(tmem, 2 * kNT);
+  (void)ok;                               // every timeout also raised sAbort
+  if (tid == 0 && *sAbort) atomicAdd(P.bad_meta, 1);
 }
 
 template <typename E, int R>
 cudaError_t shrink_tc_launch(const ShrinkArgs& a, const SegArgs& sg, lora_dtype dt,
                              cudaStream_t st, const int32_t* perm, int implicit_slots) {
+  if (sg.n_seg > kMaxSegTC) return cudaErrorNotSupported;
   ShrinkTCParams P;
   memset(&P, 0, sizeof(P));
   // row gathers need a box one row high
@@ -684,19 +968,33 @@ cudaError_t shrink_tc_launch(const ShrinkArgs& a, const SegArgs& sg, lora_dtype 
   return cudaLaunchKernelEx(&cfg, kern, P);
 }
 
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 template <typename E, int R>
 cudaError_t expand_tc_launch(const ExpandArgs& a, const SegArgs& sg, lora_dtype dt,
                              cudaStream_t st, const int32_t* perm, int implicit_slots) {
+  if (sg.n_seg > kMaxSegTC) return cudaErrorNotSupported;
   ExpandTCParams P;
   memset(&P, 0, sizeof(P));
-  int max_nt = 0;
+  long sum_nt = 0;
   for (int i = 0; i < a.n_slices; ++i) {
     cudaError_t e = encode_tmap_2d(&P.tmB[i], dt, a.B[i], (uint64_t)R,
                                    (uint64_t)a.S * a.D_out[i], (uint64_t)R * 2, R, kNT, R * 2);
     if (e != cudaSuccess) return e;
     P.y_col_off[i] = a.y_col_off[i];
     P.D_out[i] = a.D_out[i];
-    max_nt = max(max_nt, (a.D_out[i] + kNT - 1) / kNT);
+    sum_nt += (a.D_out[i] + kNT - 1) / kNT;
   }
   {
     cudaError_t e = encode_tmap_2d(&P.tmY, dt, a.y, (uint64_t)a.ldy, (uint64_t)a.T,
@@ -722,19 +1020,16 @@ cudaError_t expand_tc_launch(const ExpandArgs& a, const SegArgs& sg, lora_dtype 
   P.scale = a.scale;
   P.bad_index = const_cast<int*>(&hdr->bad_index);
   P.bad_meta = const_cast<int*>(&hdr->bad_meta);
-  const int max_tiles = (a.T + kTM - 1) / kTM + sg.n_seg;
-  // n-tiles per CTA: about three waves of one CTA per SM over all the work
-  const long units = (long)max_tiles * max_nt * a.n_slices;
-  int NJ = (int)((units + 3 * 148 - 1) / (3 * 148));
-  NJ = NJ < 1 ? 1 : (NJ > max_nt ? max_nt : NJ);
-  P.NJ = NJ;
-  P.n_chunks = (max_nt + NJ - 1) / NJ;
+  // one CTA per SM, never more CTAs than (tile, n-tile) pairs
+  const long max_tiles = (a.T + kTM - 1) / kTM + sg.n_seg;
+  const long pairs = max_tiles * sum_nt;
+  const int grid = (int)(pairs < sm_count() ? (pairs > 0 ? pairs : 1) : sm_count());
   auto kern = sgmv_expand_tc_kernel<E, R>;
   const size_t smem = ExpandSmem<R>::kTotal;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(max_tiles * P.n_chunks, a.n_slices, 1), kExpThreads, smem, st>>>(P);
+  kern<<<grid, kExpThreads, smem, st>>>(P);
   return cudaGetLastError();
 }
 
