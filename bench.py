@@ -277,10 +277,9 @@ def step_calls(p, d, what="step"):
             ops.expand_segment(buf, d.B, d.ss, d.sa, d.y, d.meta, p.scale, y_col_off=p.col_off)
         return
     if what in ("step", "fused"):
-        # the whole per-token path in one call (one launch when it fits);
-        # adapters and indices are never written by the preceding kernel here
-        ops.bgmv(d.x, d.A, d.B, d.idx, d.y, d.buf, d.meta, p.scale, y_col_off=p.col_off,
-                 pdl_early=True)
+        # the whole per-token path in one call (one launch when it fits), in
+        # plain stream order (no early start of the next launch)
+        ops.bgmv(d.x, d.A, d.B, d.idx, d.y, d.buf, d.meta, p.scale, y_col_off=p.col_off)
         return
     if what == "group":
         ops.group(d.idx, p.S, d.meta)

@@ -171,7 +171,26 @@ bgmv_fused_kernel(const __grid_constant__ FusedParams P) {
   }
   __syncthreads();
 
+  // Copies are issued in the order they are needed: the slot's A rows and the
+  // first chunk's x rows feed the shrink, B and y only the expand.  When the
+  // batch has at least two tokens per slot on average the A rows are fetched
+  // before the index scan, on the guess that this slot has tokens; a CTA whose
+  // slot turns out empty waits for them before it exits.
+  const bool spec_A = a.T >= 2 * a.S;
+  auto issue_A = [&]() {
+    if (lane == 0) {
+      const int nA = dn > 0 ? (R - warp + kFWarps - 1) / kFWarps : 0;   // rows warp, warp+8, ..
+      ptx::mbar_arrive_expect_tx(barA, (uint32_t)(max(nA, 0) * dn * 2));
+      if (dn > 0)
+        for (int j = warp; j < R; j += kFWarps)
+          ptx::bulk_g2s(sA + (size_t)j * L.pitchA, Ag + (size_t)j * D, dn * 2, barA);
+    }
+  };
   if (!a.pdl_early) ptx::grid_dep_wait();
+  // the first block of indices is requested ahead of the A rows, so that the
+  // scan does not queue behind them; each block prefetches the next
+  int v_next = tid < a.T ? a.idx[tid] : -1;
+  if (spec_A) issue_A();
 
   // 1. this slot's tokens, in token order
   int n_tok = 0;
@@ -179,7 +198,8 @@ bgmv_fused_kernel(const __grid_constant__ FusedParams P) {
   const bool counter = (unit == 0 && crank == 0);
   for (int base = 0; base < a.T; base += kFThreads) {
     const int t = base + tid;
-    int v = t < a.T ? a.idx[t] : -1;
+    const int v = v_next;
+    if (base + kFThreads < a.T) v_next = t + kFThreads < a.T ? a.idx[t + kFThreads] : -1;
     if (counter && t < a.T && (v < -1 || v >= a.S)) ++bad;
     const bool hit = (v == g);
     const unsigned bal = __ballot_sync(0xffffffffu, hit);
@@ -214,42 +234,56 @@ bgmv_fused_kernel(const __grid_constant__ FusedParams P) {
     }
   }
   ptx::grid_dep_launch_dependents();
-  if (n_tok == 0) return;   // the same for every CTA of the cluster
+  if (n_tok == 0) {                 // the same for every CTA of the cluster
+    if (spec_A && tid == 0) ptx::mbar_wait(barA, 0);   // the A rows fetched on a guess
+    return;
+  }
 
-  // 2. the slot's weights: A rows (D-chunk), B rows (output chunk); lane 0 of
-  // every warp issues its share of the copies
+  bool ok = true;
+  if (!spec_A) issue_A();
+  if (a.pdl_early) ptx::grid_dep_wait();
+  // x and y row chunks of tokens c0 .. c0+nt-1 (token k by warp k % 8)
+  auto issue_x = [&](int c0, int nt) {
+    if (lane == 0) {
+      const int nk = max((nt - warp + kFWarps - 1) / kFWarps, 0);
+      ptx::mbar_arrive_expect_tx(barX, (uint32_t)(nk * dn * 2));
+      if (dn > 0)
+        for (int k = warp; k < nt; k += kFWarps)
+          ptx::bulk_g2s(sX + (size_t)k * L.pitchA, x + (size_t)sTok[c0 + k] * a.ldx + d0, dn * 2,
+                        barX);
+    }
+  };
+  auto issue_y = [&](int c0, int nt) {
+    if (lane == 0) {
+      const int nk = max((nt - warp + kFWarps - 1) / kFWarps, 0);
+      ptx::mbar_arrive_expect_tx(barY, (uint32_t)(nk * on * 2));
+      if (on > 0)
+        for (int k = warp; k < nt; k += kFWarps)
+          ptx::bulk_g2s(sY + (size_t)k * L.pitchY, y + (size_t)sTok[c0 + k] * a.ldy + yoff, on * 2,
+                        barY);
+    }
+  };
+  // 2. the first chunk's x rows, the slot's B rows (output chunk), the first
+  // chunk's y rows; lane 0 of every warp issues its share
+  issue_x(0, min(kTB, n_tok));
   if (lane == 0) {
     const int nbox = (on + kBoxRows - 1) / kBoxRows;
-    const int nA = dn > 0 ? (R - warp + kFWarps - 1) / kFWarps : 0;     // rows warp, warp+8, ..
     const int nB = (nbox - warp + kFWarps - 1) / kFWarps;
-    ptx::mbar_arrive_expect_tx(barA, (uint32_t)(max(nA, 0) * dn * 2));
-    if (dn > 0)
-      for (int j = warp; j < R; j += kFWarps)
-        ptx::bulk_g2s(sA + (size_t)j * L.pitchA, Ag + (size_t)j * D, dn * 2, barA);
     ptx::mbar_arrive_expect_tx(barB, (uint32_t)(max(nB, 0) * L.boxBytes));
     for (int b = warp; b < nbox; b += kFWarps)
       ptx::tma_load_2d(sB + (size_t)b * L.boxBytes, &P.tmB[slice], 0,
                        g * Dout + o0 + b * kBoxRows, barB);
   }
-  if (a.pdl_early) ptx::grid_dep_wait();
+  issue_y(0, min(kTB, n_tok));
 
-  bool ok = true;
   int phase = 0;
   for (int c0 = 0; c0 < n_tok; c0 += kTB, phase ^= 1) {
     const int nt = min(kTB, n_tok - c0);
     const int NT = nt > 8 ? 2 : 1;
-    // 3a. stage this chunk's x and y row chunks (token k by warp k % 8)
-    if (lane == 0) {
-      const int nk = max((nt - warp + kFWarps - 1) / kFWarps, 0);
-      ptx::mbar_arrive_expect_tx(barX, (uint32_t)(nk * dn * 2));
-      ptx::mbar_arrive_expect_tx(barY, (uint32_t)(nk * on * 2));
-      for (int k = warp; k < nt; k += kFWarps) {
-        const int t = sTok[c0 + k];
-        if (dn > 0)
-          ptx::bulk_g2s(sX + (size_t)k * L.pitchA, x + (size_t)t * a.ldx + d0, dn * 2, barX);
-        if (on > 0)
-          ptx::bulk_g2s(sY + (size_t)k * L.pitchY, y + (size_t)t * a.ldy + yoff, on * 2, barY);
-      }
+    // 3a. this chunk's x and y row chunks (the first chunk's are on their way)
+    if (c0 > 0) {
+      issue_x(c0, nt);
+      issue_y(c0, nt);
     }
     if (c0 == 0) ok &= ptx::mbar_wait(barA, 0);
     ok &= ptx::mbar_wait(barX, phase);
@@ -310,8 +344,8 @@ bgmv_fused_kernel(const __grid_constant__ FusedParams P) {
     for (int e = tid; e < R16 * kTB; e += kFThreads) {
       float s = 0.f;
       for (int q = 0; q < CL; ++q) s += sRecv[q * R16 * kTB + e];
-      const int k = e % kTB, j = e / kTB;   // full sum over D, same in every CTA,
-      sBuf[((k >> 1) * R16 + j) * 2 + (k & 1)] = s;   // stored as token pairs
+      const int k = e % kTB, j = e / kTB;   // full sum over D, same in every CTA
+      sBuf[k * R16 + j] = s;
     }
     __syncthreads();
 
@@ -320,65 +354,108 @@ bgmv_fused_kernel(const __grid_constant__ FusedParams P) {
       float* bo = a.buf + (size_t)aslice * a.T * R;
       for (int e = tid; e < nt * R; e += kFThreads) {
         const int k = e / R, j = e % R;
-        bo[(size_t)sTok[c0 + k] * R + j] = sBuf[((k >> 1) * R16 + j) * 2 + (k & 1)];
+        bo[(size_t)sTok[c0 + k] * R + j] = sBuf[k * R16 + j];
       }
     }
 
-    // 3d. expand: thread -> CPT adjacent output columns; tokens in pairs (one
-    // packed fp32x2 accumulator per column covers two tokens).  Kept as a
-    // small runtime loop: this code runs once per CTA, so its size, not its
-    // arithmetic, sets its cost.
-    if (c0 == 0) ok &= ptx::mbar_wait(barB, 0);
-    ok &= ptx::mbar_wait(barY, phase);
+    // 3d. expand on tensor cores: y[t][o] += scale * sum_j buf[t][j] B[o][j]
+    // with mma.sync m16n8k16 (M = 16 token rows, N = 8 output columns,
+    // K = 16), so each thread's results are pairs of adjacent columns of one
+    // token: 32-bit y updates.  The fp32 intermediate enters as three
+    // bf16/fp16 terms hi + mid + lo after an exact power-of-two rescale per
+    // token: hi is buf rounded, mid the rounded remainder, lo the rounded
+    // remainder of that; both remainders are exact in fp32, so the terms carry
+    // the full fp32 value (bf16: 3 x 8 significant bits) and the products
+    // accumulate in fp32.
     {
-      constexpr int CPT = R16 <= 32 ? 2 : 1;          // columns per thread
-      using YW = typename std::conditional<CPT == 2, uint32_t, uint16_t>::type;
+      constexpr int PH = R16 * 2 + 16;                // operand row pitch (bytes)
+      char* sH = reinterpret_cast<char*>(sRed);       // [3][kTB][PH]; sRed is free here
+      float* sInvT = reinterpret_cast<float*>(sH + 3 * kTB * PH);
+      {
+        const int k = 2 * warp + (lane >> 4), li = lane & 15;   // token k, lanes of a half
+        constexpr int JL = R16 / 16;
+        float v[JL];
+        float mx = 0.f;
+#pragma unroll
+        for (int u = 0; u < JL; ++u) {
+          v[u] = k < nt ? sBuf[k * R16 + li + 16 * u] : 0.f;
+          mx = fmaxf(mx, fabsf(v[u]));
+        }
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        int ex = ((__float_as_int(mx) >> 23) & 0xff) - 127;
+        ex = (mx > 0.f && ex > -100 && ex < 100) ? ex : 0;
+        const float sc = __int_as_float((127 - ex + 7) << 23);
+        if (li == 0) sInvT[k] = __int_as_float((127 + ex - 7) << 23);
+#pragma unroll
+        for (int u = 0; u < JL; ++u) {
+          const float w0 = v[u] * sc;
+          const uint16_t h0 = Elem<E>::from_f32(w0);
+          const float w1 = w0 - Elem<E>::to_f32(h0);
+          const uint16_t h1 = Elem<E>::from_f32(w1);
+          const uint16_t h2 = Elem<E>::from_f32(w1 - Elem<E>::to_f32(h1));
+          char* row = sH + k * PH + (li + 16 * u) * 2;
+          *reinterpret_cast<uint16_t*>(row) = h0;
+          *reinterpret_cast<uint16_t*>(row + kTB * PH) = h1;
+          *reinterpret_cast<uint16_t*>(row + 2 * kTB * PH) = h2;
+        }
+      }
+      if (c0 == 0) ok &= ptx::mbar_wait(barB, 0);
+      ok &= ptx::mbar_wait(barY, phase);
+      __syncthreads();
+      // A fragments (token rows) of the three terms; B fragments: output rows
+      const uint32_t aBase = ptx::smem_u32(sH) + (lane & 15) * PH + (lane >> 4) * 16;
+      const int t0 = lane >> 2;                        // this thread's token rows t0, t0 + 8
+      const float inv0 = sInvT[t0], inv1 = sInvT[t0 + 8];
+      char* yrow0 = sY + (size_t)t0 * L.pitchY + 4 * (lane & 3);
+      char* yrow1 = yrow0 + 8 * (size_t)L.pitchY;
+      const bool row0 = t0 < nt, row1 = NT == 2 && t0 + 8 < nt;
+      const int MTo = (on + 15) / 16;
 #pragma unroll 1
-      for (int o = tid * CPT; o < on; o += kFThreads * CPT) {
-        uint64_t bd[CPT][R16];                        // (B[o][j], B[o][j])
+      for (int mt = warp; mt < MTo; mt += kFWarps) {
+        float acc[2][4];
 #pragma unroll
-        for (int c = 0; c < CPT; ++c) {
-          const int oc = o + c;
-          const int box = oc / kBoxRows, rb = oc % kBoxRows;
-          const char* brow = sB + (size_t)box * L.boxBytes + (size_t)rb * (R16 * 2);
+        for (int n = 0; n < 2; ++n)
 #pragma unroll
-          for (int q = 0; q < R16 / 8; ++q) {
-            float f[8];
-            Elem<E>::to_f32(*reinterpret_cast<const uint4*>(brow + swz_chunk<R16>(rb, q) * 16), f);
+          for (int q = 0; q < 4; ++q) acc[n][q] = 0.f;
+        // B rows mt*16 + 0..15: lanes 0-15 the first 8 rows (k chunks 0/1),
+        // lanes 16-31 the next 8
+        const int orow = mt * 16 + (lane & 7) + 8 * (lane >> 4);
+        const char* brow = sB + (size_t)(orow / kBoxRows) * L.boxBytes +
+                           (size_t)(orow % kBoxRows) * (R16 * 2);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) bd[c][q * 8 + u] = ptx::pack2(f[u], f[u]);
+        for (int ks = 0; ks < R16 / 16; ++ks) {
+          uint32_t bf[4];
+          ptx::ldsm_x4(ptx::smem_u32(brow + swz_chunk<R16>(orow % kBoxRows,
+                                                           2 * ks + ((lane >> 3) & 1)) * 16),
+                       bf[0], bf[1], bf[2], bf[3]);
+#pragma unroll
+          for (int term = 0; term < 3; ++term) {
+            uint32_t af[4];
+            ptx::ldsm_x4(aBase + term * kTB * PH + ks * 32, af[0], af[1], af[2], af[3]);
+            ptx::mma_16816<kBF>(acc[0], af, bf[0], bf[1]);
+            ptx::mma_16816<kBF>(acc[1], af, bf[2], bf[3]);
           }
         }
-#pragma unroll 1
-        for (int k = 0; k < nt; k += 2) {
-          const float2* bp = reinterpret_cast<const float2*>(sBuf) + (k >> 1) * R16;
-          uint64_t acc[CPT][2];
+        // acc[n][0..1]: token t0, columns o, o+1 with o = 16 mt + 8n + 2 (lane%4);
+        // acc[n][2..3]: token t0 + 8
 #pragma unroll
-          for (int c = 0; c < CPT; ++c) acc[c][0] = acc[c][1] = 0;
-#pragma unroll
-          for (int j = 0; j < R16; ++j) {
-            const float2 v = bp[j];                   // (buf[k][j], buf[k+1][j]), broadcast
-            const uint64_t av = ptx::pack2(v.x, v.y);
-#pragma unroll
-            for (int c = 0; c < CPT; ++c) acc[c][j & 1] = ptx::ffma2(av, bd[c][j], acc[c][j & 1]);
+        for (int n = 0; n < 2; ++n) {
+          const int o = mt * 16 + 8 * n + 2 * (lane & 3);
+          if (o < on) {                               // on is a multiple of 8
+            uint32_t* p0 = reinterpret_cast<uint32_t*>(yrow0 + (mt * 16 + 8 * n) * 2);
+            uint32_t* p1 = reinterpret_cast<uint32_t*>(yrow1 + (mt * 16 + 8 * n) * 2);
+            const uint32_t w0 = row0 ? *p0 : 0u;
+            const uint32_t w1 = row1 ? *p1 : 0u;
+            const uint16_t* h0 = reinterpret_cast<const uint16_t*>(&w0);
+            const uint16_t* h1 = reinterpret_cast<const uint16_t*>(&w1);
+            if (row0)
+              *p0 = Elem<E>::pack2(fmaf(a.scale, acc[n][0] * inv0, Elem<E>::to_f32(h0[0])),
+                                   fmaf(a.scale, acc[n][1] * inv0, Elem<E>::to_f32(h0[1])));
+            if (row1)
+              *p1 = Elem<E>::pack2(fmaf(a.scale, acc[n][2] * inv1, Elem<E>::to_f32(h1[0])),
+                                   fmaf(a.scale, acc[n][3] * inv1, Elem<E>::to_f32(h1[1])));
           }
-          YW* y0 = reinterpret_cast<YW*>(sY + (size_t)k * L.pitchY + o * 2);
-          YW* y1 = reinterpret_cast<YW*>(sY + (size_t)(k + 1) * L.pitchY + o * 2);
-          const YW w0 = *y0;
-          const YW w1 = (k + 1 < nt) ? *y1 : w0;
-          YW r0, r1;
-#pragma unroll
-          for (int c = 0; c < CPT; ++c) {
-            const uint64_t t = acc[c][0];
-            const uint64_t u = acc[c][1];
-            const float s0 = ptx::lo32(t) + ptx::lo32(u), s1 = ptx::hi32(t) + ptx::hi32(u);
-            reinterpret_cast<uint16_t*>(&r0)[c] = Elem<E>::from_f32(
-                fmaf(a.scale, s0, Elem<E>::to_f32(reinterpret_cast<const uint16_t*>(&w0)[c])));
-            reinterpret_cast<uint16_t*>(&r1)[c] = Elem<E>::from_f32(
-                fmaf(a.scale, s1, Elem<E>::to_f32(reinterpret_cast<const uint16_t*>(&w1)[c])));
-          }
-          *y0 = r0;
-          if (k + 1 < nt) *y1 = r1;
         }
       }
     }

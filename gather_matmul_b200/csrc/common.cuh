@@ -72,6 +72,11 @@ template <> struct Elem<__half> {
   static __device__ __forceinline__ uint16_t from_f32(float f) {
     return __half_as_ushort(__float2half_rn(f));
   }
+  // two floats -> two packed halves (round to nearest even), a in the low half
+  static __device__ __forceinline__ uint32_t pack2(float a, float b) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
 };
 template <> struct Elem<__nv_bfloat16> {
   static __device__ __forceinline__ void to_f32(const uint4& v, float* f) {
@@ -87,6 +92,10 @@ template <> struct Elem<__nv_bfloat16> {
   }
   static __device__ __forceinline__ uint16_t from_f32(float f) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+  }
+  static __device__ __forceinline__ uint32_t pack2(float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
   }
 };
 

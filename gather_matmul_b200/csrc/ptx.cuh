@@ -235,6 +235,14 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
 }
 // 32 lanes x 32 bits, 16 consecutive columns: thread i of the warp gets TMEM
 // lane (warp quadrant base + i), columns [col, col + 16).
+// 32 lanes x 8 consecutive 32-bit TMEM columns: r[i] = column base + i of
+// this thread's lane.
+__device__ __forceinline__ void tc_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
 __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"

@@ -46,7 +46,6 @@ constexpr int kTM = 128;          // token rows per tile (MMA M)
 constexpr int kBK = 64;           // K elements per pipeline stage: one 128-byte row
 template <int R>
 constexpr int stages_for() { return R <= 32 ? 6 : 4; }   // two CTAs per SM at every rank
-constexpr int kThreads = 128;     // 4 warps: one per 32 TMEM lanes
 constexpr int kNT = 128;          // expand output columns per CTA (MMA N)
 
 struct TileInfo {
@@ -402,10 +401,11 @@ struct ExpandSmem {
 };
 
 // Bytes a pair moves, in units the schedule balances: the B tile, the valid
-// y rows read and written, and a fixed per-pair cost.
+// y rows read and written, and a fixed per-pair cost (the pipeline time of a
+// pair that moves almost nothing, in bytes at one SM's share of HBM bandwidth).
 template <int R>
 __device__ __forceinline__ int64_t pair_weight(int valid) {
-  return (int64_t)kNT * R * 2 + 512 * (int64_t)valid + 4096;
+  return (int64_t)kNT * R * 2 + 512 * (int64_t)valid + 16384;
 }
 
 struct SegView {
@@ -583,9 +583,13 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   }
 
   if (warp == kExpMma) {
-    // this CTA's share of the weighted pair sequence
+    ptx::tmem_alloc(tmem_slot, 2 * kNT);
+    ptx::tmem_relinquish();
+    // this CTA's share of the weighted pair sequence (the segment reads stay in
+    // bounds whatever the workspace holds, so they need not wait for the check)
+    const int64_t Wt0 = seg_chunk_weights<R>(sv, chunkW);
     const bool meta_ok = !P.implicit_slots || grouped_meta_ok(P.bad_index, P.T, P.S, lane == 0);
-    const int64_t Wt = meta_ok ? seg_chunk_weights<R>(sv, chunkW) : 0;
+    const int64_t Wt = meta_ok ? Wt0 : 0;
     const int64_t W = Wt * sum_nt;
     if (lane == 0) {
       sRange[0] = W * (int64_t)blockIdx.x / gridDim.x;
@@ -593,8 +597,6 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
       sRange[2] = Wt;
     }
     __syncwarp();
-    ptx::tmem_alloc(tmem_slot, 2 * kNT);
-    ptx::tmem_relinquish();
   }
   if (tid == 0) {
     *sAbort = 0;
@@ -805,18 +807,28 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
               for (int k = 0; k < 4; ++k) ptx::tc_ld16(tacc + 64 * h + 16 * k, r + 16 * k);
               ptx::tc_wait_ld();
               if (m < rn.valid) {
+                // all eight 16-byte pieces of the row first, then the math, then
+                // the stores (the loads must not wait behind earlier stores)
                 char* row = ys + h * L::kYHalf + m * 128;
+                uint4 w[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                  w[c] = *reinterpret_cast<const uint4*>(row + ((c ^ (m & 7)) << 4));
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                  uint4* pc = reinterpret_cast<uint4*>(row + ((c ^ (m & 7)) << 4));
-                  uint4 w = *pc;
-                  uint16_t* hw = reinterpret_cast<uint16_t*>(&w);
+                  float f[8];
+                  Elem<E>::to_f32(w[c], f);
+                  uint32_t o[4];
 #pragma unroll
-                  for (int v = 0; v < 8; ++v)
-                    hw[v] = Elem<E>::from_f32(fmaf(P.scale, __uint_as_float(r[8 * c + v]) * inv,
-                                                   Elem<E>::to_f32(hw[v])));
-                  *pc = w;
+                  for (int v = 0; v < 4; ++v)
+                    o[v] = Elem<E>::pack2(
+                        fmaf(P.scale, __uint_as_float(r[8 * c + 2 * v]) * inv, f[2 * v]),
+                        fmaf(P.scale, __uint_as_float(r[8 * c + 2 * v + 1]) * inv, f[2 * v + 1]));
+                  w[c] = make_uint4(o[0], o[1], o[2], o[3]);
                 }
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                  *reinterpret_cast<uint4*>(row + ((c ^ (m & 7)) << 4)) = w[c];
               }
             }
             ptx::tc_fence_before();
@@ -835,53 +847,76 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
                 deferred = s;
               }
             } else {
-              // rows 32q .. 32q+31 of half h: lane -> (row 4i + lane / 8, chunk lane % 8)
-#pragma unroll 2
+              // rows 32q .. 32q+31 of half h: lane -> (row 4i + lane / 8, chunk lane % 8);
+              // all shared-memory reads first, then the global stores
+              const int ch = lane & 7;
+              const bool col_ok = 64 * h + 8 * ch < nn;
+              uint4 v[8];
+#pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const int lr = 4 * i + (lane >> 3), ch = lane & 7;
-                const int mr = q * 32 + lr;
+                const int mr = q * 32 + 4 * i + (lane >> 3);
+                v[i] = *reinterpret_cast<const uint4*>(ys + h * L::kYHalf + mr * 128 +
+                                                       ((ch ^ (mr & 7)) << 4));
+              }
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const int lr = 4 * i + (lane >> 3);
                 const int tk = __shfl_sync(0xffffffffu, tok, lr);
-                if (mr < rn.valid && 64 * h + 8 * ch < nn) {
-                  const uint4 v = *reinterpret_cast<const uint4*>(
-                      ys + h * L::kYHalf + mr * 128 + ((ch ^ (mr & 7)) << 4));
-                  *reinterpret_cast<uint4*>(ycol + (size_t)tk * P.ldy + n0 + 64 * h + 8 * ch) = v;
-                }
+                if (q * 32 + lr < rn.valid && col_ok)
+                  *reinterpret_cast<uint4*>(ycol + (size_t)tk * P.ldy + n0 + 64 * h + 8 * ch) = v[i];
               }
               ptx::fence_proxy_async_smem();
             }
           } else {
-            // swapped: thread = output column 32q + lane; token chunks of 16
+            // swapped: thread = output column 32q + lane; groups of 8 tokens
             // alternate between the two warps of the quadrant
             const int col = q * 32 + lane;
             const int hc = col >> 6, cc = col & 63;
             char* cbase = ys + hc * L::kYHalf + (cc & 7) * 2;
-            const int nch = (rn.valid + 15) / 16;
-            for (int k = h; k < nch; k += 2) {
-              uint32_t r[16];
-              ptx::tc_ld16(tacc + 16 * k, r);
+            const int ng = (rn.valid + 7) / 8;
+            for (int g = h; g < ng; g += 2) {
+              uint32_t r[8];
+              ptx::tc_ld8(tacc + 8 * g, r);
+              const float4 i0 = *reinterpret_cast<const float4*>(invs + 8 * g);
+              const float4 i1 = *reinterpret_cast<const float4*>(invs + 8 * g + 4);
+              const float iv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+              // token t = 8g + v sits in row t, whose swizzle phase is t & 7 = v
+              uint16_t* py[8];
+              uint16_t yv[8];
+#pragma unroll
+              for (int v = 0; v < 8; ++v) {
+                py[v] = reinterpret_cast<uint16_t*>(cbase + (8 * g + v) * 128 +
+                                                    (((cc >> 3) ^ v) << 4));
+                yv[v] = *py[v];
+              }
               ptx::tc_wait_ld();
 #pragma unroll
-              for (int v = 0; v < 16; ++v) {
-                const int t = 16 * k + v;
-                if (t < rn.valid) {
-                  uint16_t* py = reinterpret_cast<uint16_t*>(cbase + t * 128 + (((cc >> 3) ^ (t & 7)) << 4));
-                  *py = Elem<E>::from_f32(
-                      fmaf(P.scale, __uint_as_float(r[v]) * invs[t], Elem<E>::to_f32(*py)));
-                }
-              }
+              for (int v = 0; v < 8; ++v)
+                if (8 * g + v < rn.valid)
+                  *py[v] = Elem<E>::from_f32(
+                      fmaf(P.scale, __uint_as_float(r[v]) * iv[v], Elem<E>::to_f32(yv[v])));
             }
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&accempty[a]);
             asm volatile("bar.sync 3, 256;" ::: "memory");   // every column of every row done
-            // rows 0 .. valid-1, 16 chunks each: e -> (row e / 16, chunk e % 16)
-            for (int e = warp * 32 + lane; e < rn.valid * 16; e += 256) {
+            // rows 0 .. valid-1, 16 chunks each: e -> (row e / 16, chunk e % 16);
+            // at most 64 rows: four pieces per thread, all read before any store
+            uint4 v[4];
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int e = warp * 32 + lane + 256 * it;
+              const int mr = min(e >> 4, kSwapMax - 1), hh = (e >> 3) & 1, ch = e & 7;
+              v[it] = *reinterpret_cast<const uint4*>(ys + hh * L::kYHalf + mr * 128 +
+                                                      ((ch ^ (mr & 7)) << 4));
+            }
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int e = warp * 32 + lane + 256 * it;
               const int mr = e >> 4, hh = (e >> 3) & 1, ch = e & 7;
-              if (64 * hh + 8 * ch < nn) {
-                const uint4 v = *reinterpret_cast<const uint4*>(
-                    ys + hh * L::kYHalf + mr * 128 + ((ch ^ (mr & 7)) << 4));
-                *reinterpret_cast<uint4*>(ycol + (size_t)toks[mr] * P.ldy + n0 + 64 * hh + 8 * ch) = v;
-              }
+              if (mr < rn.valid && 64 * hh + 8 * ch < nn)
+                *reinterpret_cast<uint4*>(ycol + (size_t)toks[mr] * P.ldy + n0 + 64 * hh + 8 * ch) =
+                    v[it];
             }
             ptx::fence_proxy_async_smem();
           }
