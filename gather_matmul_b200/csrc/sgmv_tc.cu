@@ -950,6 +950,19 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   if (tid == 0 && *sAbort) atomicAdd(P.bad_meta, 1);
 }
 
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 template <typename E, int R>
 cudaError_t shrink_tc_launch(const ShrinkArgs& a, const SegArgs& sg, lora_dtype dt,
                              cudaStream_t st, const int32_t* perm, int implicit_slots) {
@@ -980,14 +993,36 @@ cudaError_t shrink_tc_launch(const ShrinkArgs& a, const SegArgs& sg, lora_dtype 
   P.bad_meta = const_cast<int*>(&hdr->bad_meta);
   const int max_tiles = (a.T + kTM - 1) / kTM + sg.n_seg;
   const int nkb_all = (a.D + kBK - 1) / kBK;
-  // split K across a cluster when there are too few tiles to fill the GPU
+  // split K across a cluster when there are too few tiles to fill the GPU:
+  // up to 16 ranks (a non-portable cluster size, used when the device takes it)
+  const int nsm = sm_count();
   int KS = 1;
-  while (KS < 4 && (long)max_tiles * a.n_slices * KS < 148 && nkb_all >= 4 * KS) KS *= 2;
-  P.KS = KS;
+  while (KS < 16 && (long)max_tiles * a.n_slices * KS < nsm && nkb_all >= 4 * KS) KS *= 2;
   auto kern = sgmv_shrink_tc_kernel<E, R>;
   const size_t smem = ShrinkSmem<R>::kTotal;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  if (KS == 16) {
+    int active = 0;
+    cudaLaunchConfig_t q = {};
+    q.gridDim = dim3(16, 1, 1);
+    q.blockDim = dim3(kShrThreads, 1, 1);
+    q.dynamicSmemBytes = smem;
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = 16;
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    q.attrs = qa;
+    q.numAttrs = 1;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&active, kern, &q) != cudaSuccess || active < 1) {
+      cudaGetLastError();
+      KS = 8;
+    }
+  }
+  P.KS = KS;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(max_tiles * KS, a.n_slices, 1);
   cfg.blockDim = dim3(kShrThreads, 1, 1);
@@ -1001,19 +1036,6 @@ cudaError_t shrink_tc_launch(const ShrinkArgs& a, const SegArgs& sg, lora_dtype 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, P);
-}
-
-int sm_count() {
-  static int cache[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-    cache[dev] = n;
-  }
-  return cache[dev];
 }
 
 template <typename E, int R>

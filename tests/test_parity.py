@@ -87,3 +87,40 @@ def test_sgmv_segments(case):
     p = W.make_problem("segments", dt, T=T, D=D, r=r, S=S, d_out=d_out, scale=1.25,
                        seed=len(ss) * 7 + D, segments=(np.array(ss), np.array(sa)))
     _run_and_check(p)
+
+
+def _many_segments(n_seg, seg_len, S, every_neg):
+    ss = np.arange(n_seg + 1, dtype=np.int64) * seg_len
+    sa = np.array([-1 if (i % every_neg) == every_neg - 1 else i % S for i in range(n_seg)])
+    return ss, sa
+
+
+def test_sgmv_many_tiles_per_cta():
+    """2048 segments of 8 tokens over 8 output slices of 128 columns: about
+    a hundred tile runs per CTA of the persistent expand, more than one run
+    list holds, so the lists are rebuilt mid-kernel."""
+    ss, sa = _many_segments(2048, 8, 16, 7)
+    p = W.make_problem("many_tiles", W.BF16, T=int(ss[-1]), D=64, r=16, S=16,
+                       d_out=[128] * 8, scale=0.75, seed=11, segments=(ss, sa))
+    _run_and_check(p)
+
+
+def test_sgmv_long_segment_list_item_kernels():
+    """More than 2048 segments: the segment calls take the item kernels."""
+    ss, sa = _many_segments(2050, 2, 5, 4)
+    p = W.make_problem("long_list", W.F16, T=int(ss[-1]), D=256, r=32, S=5,
+                       d_out=[256], scale=1.5, seed=12, segments=(ss, sa))
+    _run_and_check(p)
+
+
+def test_sgmv_many_mixed_segments():
+    """Forty segments of mixed lengths (1 to 513 tokens, some without an
+    adapter, adapters repeated): more tiles than the GPU has SMs, full and
+    partial tiles interleaved."""
+    rng = np.random.default_rng(13)
+    lens = rng.choice([1, 37, 128, 200, 256, 300, 513], size=40)
+    ss = np.concatenate([[0], np.cumsum(lens)])
+    sa = rng.integers(-1, 6, size=40)
+    p = W.make_problem("mixed_segments", W.BF16, T=int(ss[-1]), D=1024, r=32, S=6,
+                       d_out=[512], scale=0.5, seed=13, segments=(ss, sa))
+    _run_and_check(p)
