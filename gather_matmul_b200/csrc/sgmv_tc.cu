@@ -236,7 +236,17 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
       perm ? (uint32_t)(ngroups * 4 * 128 + L::kABytes) : (uint32_t)L::kStageBytes;
   if (warp < 4) {
     // load warps: the adapter tile and the x tile (one 2-D tile, or up to 32
-    // four-row gathers, gather g issued by warp g % 4, lane g / 4)
+    // four-row gathers, gather g issued by warp g % 4, lane g / 4); a gather's
+    // four token rows are the same at every K step, so they are read once
+    const int g = warp + 4 * lane;
+    int rr[4] = {0, 0, 0, 0};
+    if (perm && g < ngroups) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int p = m0 + 4 * g + j;
+        rr[j] = perm[p < m0 + valid ? p : m0];
+      }
+    }
     for (int i = 0; i < nkb; ++i) {
       const int s = i % kStages;
       const uint32_t ph = (i / kStages) & 1;
@@ -254,16 +264,8 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
         }
       }
       __syncwarp();
-      const int g = warp + 4 * lane;
-      if (perm && g < ngroups) {
-        int rr[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int p = m0 + 4 * g + j;
-          rr[j] = perm[p < m0 + valid ? p : m0];
-        }
+      if (perm && g < ngroups)
         ptx::tma_gather4(st + g * 4 * 128, &P.tmX, kx, rr[0], rr[1], rr[2], rr[3], &full[s]);
-      }
     }
   } else if (lane == 0) {
     // MMA issuer (warp 4)
