@@ -11,29 +11,34 @@
 //      host round trip ("[Hardware][TPU][V1] Better tpu multilora
 //      compilation": indices moved to the device; the per-token gather the
 //      PyTorch baseline paid for is replaced by one read of each adapter);
-//   2. the slot's A rows (its D-chunk) and B rows (its output chunk) are staged
-//      in shared memory with bulk / TMA copies, once for all its tokens;
-//   3. per chunk of <= 16 tokens: the tokens' x and y row chunks are staged;
-//      shrink partials buf^T[r x tok] = A[r x Dc] x^T[Dc x tok] run on tensor
-//      cores (mma.sync m16n8k16, bf16/fp16 in, fp32 accumulate) with the
-//      tokens as the narrow n=8 side, so a decode slot of 8 tokens wastes no
-//      tensor work; warps split the K range and add their fragments in a
-//      fixed order; the CL partials are summed in rank order through
-//      distributed shared memory, so every CTA holds the full fp32 buf rows
-//      (no atomics, no pre-zeroed intermediate, bitwise reproducible);
-//   4. expand y[tok][o] += scale * sum_j buf[tok][j] B[o][j] on CUDA cores in
-//      fp32 with packed two-lane FMAs (fma.rn.f32x2): the intermediate is kept
-//      as token pairs so one 64-bit operand carries two tokens, and each B
-//      value is duplicated into both lanes once per column.  The intermediate
-//      is used at full fp32 precision, never reduced to half ("Add multi-LoRA
-//      support", Limitations list on the SGMV intermediate).  Each thread owns
-//      one or two output columns and runs four independent accumulator chains;
-//      y is updated in shared memory with one fp32 fma and one
-//      round-to-nearest-even, then written back with coalesced 16-byte stores.
+//   2. the copies are issued in the order they are needed: the slot's A rows
+//      (its D-chunk; fetched before the scan when the batch averages two or
+//      more tokens per slot) and the first chunk's x rows feed the shrink, the
+//      B rows (its output chunk, by TMA) and y rows only the expand, so the
+//      shrink starts while the expand's operands are still streaming in;
+//   3. per chunk of <= 16 tokens: shrink partials buf^T[r x tok] =
+//      A[r x Dc] x^T[Dc x tok] run on tensor cores (mma.sync m16n8k16,
+//      bf16/fp16 in, fp32 accumulate) with the tokens as the narrow n = 8
+//      side, so a decode slot of 8 tokens wastes no tensor work; warps split
+//      the K range and add their fragments in a fixed order; the CL partials
+//      are summed in rank order through distributed shared memory, so every
+//      CTA holds the full fp32 buf rows (no atomics, no pre-zeroed
+//      intermediate, bitwise reproducible);
+//   4. expand y[tok][o] += scale * sum_j buf[tok][j] B[o][j] on tensor cores
+//      (mma.sync m16n8k16 with the tokens as M and 8 output columns as N, so
+//      each thread updates adjacent column pairs of one token).  The fp32
+//      intermediate enters as three half-precision terms hi + mid + lo after
+//      an exact power-of-two rescale per token; the remainders are exact in
+//      fp32, so the terms carry each value to about 2^-24 of the token's
+//      largest one (bf16: three 8-bit significands) and the products
+//      accumulate in fp32: it is never reduced to half precision ("Add
+//      multi-LoRA support", Limitations list on the SGMV intermediate).  y is
+//      updated in shared memory with one fp32 fma and one round-to-nearest-
+//      even, then written back with coalesced 16-byte stores.
 //
 // Launched with programmatic dependent launch: the next kernel in the stream
 // may start its own prologue while this one runs; with pdl_early the slot's
-// weights and the indices are read before waiting for the previous kernel.
+// A rows and the indices are read before waiting for the previous kernel.
 // Every wait on an mbarrier is bounded; a timeout is counted in the workspace
 // and the kernel finishes its cluster barriers without hanging.
 #include <cooperative_groups.h>

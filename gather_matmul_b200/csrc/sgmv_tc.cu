@@ -10,21 +10,24 @@
 //
 // Shrink  buf[rows][:] = X[rows][:] . A[a]^T     M = 128 tokens, N = r, K = D
 //   One CTA per (128-row tile of a segment, K-split); a cluster of KS CTAs
-//   covers the K range of one tile.  A 4-6 stage pipeline of 64-wide K blocks:
-//   TMA loads the x tile (128 x 64, 128-byte swizzle) and the adapter tile
-//   (r x 64); one thread issues tcgen05.mma (kind::f16, fp32 accumulator in
-//   tensor memory) and tcgen05.commit frees the stage.  The accumulator is read
-//   back with tcgen05.ld; split-K partials are summed in rank order through
-//   distributed shared memory (deterministic, no atomics).
+//   (up to 16) covers the K range of one tile when tiles are too few to fill
+//   the GPU.  A 4-6 stage pipeline of 64-wide K blocks: four load warps (one
+//   per SM sub-partition) bring the adapter tile (r x 64) and the x tile
+//   (128 x 64, 128-byte swizzle) by TMA, as one 2-D box for consecutive rows
+//   or as 4-row gathers (tile::gather4) through the grouping permutation; one
+//   thread issues tcgen05.mma (kind::f16, fp32 accumulator in tensor memory)
+//   and tcgen05.commit frees the stage.  The accumulator is read back with
+//   tcgen05.ld; split-K partials are pushed to the owning rank through
+//   distributed shared memory and summed in rank order (no atomics).
 // Expand  Y[rows][cols] += scale * buf[rows][:] . B[a][cols]^T   M = 128, N = 128, K = r
-//   One CTA per (tile, 128 output columns, slice).  The fp32 intermediate
-//   enters the tensor core as hi + lo of the input type after an exact
-//   power-of-two rescale per row (about 16 bits for bf16, 22 for fp16), two
-//   MMAs per K step into one fp32 accumulator.  The B tile arrives by TMA;
-//   each thread prefetches its row's y values into registers at the start
-//   (whole 32-byte sectors), so four CTAs fit per SM; the epilogue adds
-//   scale * acc with one round-to-nearest-even and stores from registers.
-//   Rows past the segment are never written.
+//   Persistent, one CTA per SM over a byte-weighted static schedule of
+//   (slice, tile, 128-column) pairs (see the expand section below).  The fp32
+//   intermediate enters the tensor core as hi + lo of the input type after an
+//   exact power-of-two rescale per row (about 16 bits for bf16, 22 for fp16),
+//   two MMAs per K step into one fp32 accumulator; a tile of at most 64 rows
+//   swaps the operands.  y tiles move by 2-D TMA (consecutive rows) or 4-row
+//   gathers; the epilogue adds scale * acc with one round-to-nearest-even.
+//   Rows past the segment and rows without an adapter are never written.
 //
 // Every mbarrier wait is bounded (about one second); a timeout is counted in
 // the workspace and the kernel still releases its tensor memory and exits.
