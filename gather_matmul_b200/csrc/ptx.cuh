@@ -34,6 +34,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+// A waiting thread is suspended in mbarrier.try_wait until the phase completes
+// or this many nanoseconds pass, instead of spinning on the issue slots that
+// other warps of the SM need.
+constexpr uint32_t kWaitSuspendNs = 1000000;
+
 // Wait for the phase with the given parity to complete.  Gives up after
 // about one second and returns false (the caller records an error and stops
 // instead of hanging the GPU).
@@ -43,10 +48,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   for (uint32_t it = 0;; ++it) {
     uint32_t ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
         " selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(addr), "r"(parity)
+        : "r"(addr), "r"(parity), "r"(kWaitSuspendNs)
         : "memory");
     if (ok) return true;
     if (it == 0) t0 = globaltimer_ns();
@@ -64,10 +69,10 @@ __device__ __forceinline__ bool mbar_wait_ff(uint64_t* bar, uint32_t parity, vol
   for (uint32_t it = 0;; ++it) {
     uint32_t ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
         " selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(addr), "r"(parity)
+        : "r"(addr), "r"(parity), "r"(kWaitSuspendNs)
         : "memory");
     if (ok) return true;
     if ((it & 63) == 0) {
