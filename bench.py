@@ -40,6 +40,7 @@ from gather_matmul_b200 import workloads as W  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "gather_matmul_b200", "csrc", f)
                   for f in ("bgmv.cu", "bgmv_fused.cu", "group.cu", "sgmv_tc.cu", "common.cuh",
@@ -107,6 +108,16 @@ def measured_peaks():
         d = json.load(open(path))
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_bf16_tflops():
+    """Dense bf16 tensor peak (burst cuBLAS GEMM) of this machine's B200s."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"])
+    return FALLBACK_BF16_TFLOPS
 
 
 def profile_traffic(kernel):
@@ -558,6 +569,7 @@ def run_ours(args):
 def detail_all(args, stream, peak, peak_kind):
     """Per-projection numbers of every workload (not the headline line)."""
     out = {}
+    tf_peak = measured_bf16_tflops()
     for n in (1, 2, 3, 4, 5):
         for p in W.config(n):
             sets = make_sets(p, extra_copies=True)
@@ -580,6 +592,11 @@ def detail_all(args, stream, peak, peak_kind):
                 "kernel_frac": {k: round(kernel_bytes(p, k) / v / 1e9 / peak, 4)
                                 for k, v in kt.items()},
                 "tflops_step": round(fl / t / 1e12, 2),
+                # fraction of the tensor roofline, and of the slower of the two
+                # rooflines (contraction FLOPs at the bf16 peak, bytes at HBM)
+                "tensor_frac_step": round(fl / t / 1e12 / tf_peak, 4),
+                "roofline_frac_step": round(max(fl / (tf_peak * 1e12), by["step"] / (peak * 1e9))
+                                            / t, 4),
                 "bytes": by,
             }
             del sets
