@@ -361,42 +361,65 @@ def make_sets(p, extra_copies):
     return sets
 
 
-def e2e_measure(p, d, steps, warmup, stream):
+def e2e_measure(p, dsets, steps, warmup, stream):
     """The same metric through the public API with host buffers: per step,
-    pinned host -> device copies of x, idx and y, the three calls, and a
-    device -> host copy of the updated y."""
-    hx = torch.empty(d.x.shape, dtype=d.x.dtype, pin_memory=True)
-    hy = torch.empty(d.y.shape, dtype=d.y.dtype, pin_memory=True)
-    hout = torch.empty(d.y.shape, dtype=d.y.dtype, pin_memory=True)
-    hx.copy_(d.x.cpu())
-    hy.copy_(d.y.cpu())
+    pinned host -> device copies of x, idx and y, the call(s), and a device ->
+    host copy of the updated y.  Steps are double-buffered over two device
+    sets and three streams (copy in, compute, copy out), as a serving loop
+    would overlap one batch's transfers with another's compute; every step
+    still moves all of its bytes across PCIe."""
+    nb = min(2, len(dsets))
+    dsets = dsets[:nb]
+    d0 = dsets[0]
+    hx = torch.empty(d0.x.shape, dtype=d0.x.dtype, pin_memory=True)
+    hy = torch.empty(d0.y.shape, dtype=d0.y.dtype, pin_memory=True)
+    hout = [torch.empty(d0.y.shape, dtype=d0.y.dtype, pin_memory=True) for _ in range(nb)]
+    hx.copy_(d0.x.cpu())
+    hy.copy_(d0.y.cpu())
     hidx = None
-    if d.idx is not None:
-        hidx = torch.empty(d.idx.shape, dtype=d.idx.dtype, pin_memory=True)
-        hidx.copy_(d.idx.cpu())
+    if d0.idx is not None:
+        hidx = torch.empty(d0.idx.shape, dtype=d0.idx.dtype, pin_memory=True)
+        hidx.copy_(d0.idx.cpu())
     h2d = hx.numel() * hx.element_size() + hy.numel() * hy.element_size() + \
         (hidx.numel() * 4 if hidx is not None else 0)
-    d2h = hout.numel() * hout.element_size()
+    d2h = hout[0].numel() * hout[0].element_size()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    done_in = [torch.cuda.Event() for _ in range(nb)]
+    done_step = [torch.cuda.Event() for _ in range(nb)]
+    done_out = [torch.cuda.Event() for _ in range(nb)]
+    used = [False] * nb
 
-    def one():
-        d.x.copy_(hx, non_blocking=True)
-        d.y.copy_(hy, non_blocking=True)
-        if hidx is not None:
-            d.idx.copy_(hidx, non_blocking=True)
-        step_calls(p, d)
-        hout.copy_(d.y, non_blocking=True)
+    def one(k):
+        i = k % nb
+        d = dsets[i]
+        with torch.cuda.stream(s_in):
+            if used[i]:
+                s_in.wait_event(done_out[i])          # set i's previous result has left
+            d.x.copy_(hx, non_blocking=True)
+            d.y.copy_(hy, non_blocking=True)
+            if hidx is not None:
+                d.idx.copy_(hidx, non_blocking=True)
+            done_in[i].record(s_in)
+        with torch.cuda.stream(stream):
+            stream.wait_event(done_in[i])
+            step_calls(p, d)
+            done_step[i].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done_step[i])
+            hout[i].copy_(d.y, non_blocking=True)
+            done_out[i].record(s_out)
+        used[i] = True
 
-    with torch.cuda.stream(stream):
-        for _ in range(warmup):
-            one()
+    for k in range(warmup):
+        one(k)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(steps):
-            one()
-    e1.record(stream)
+    e0.record(s_in)
+    for k in range(steps):
+        one(k)
+    s_out.wait_event(done_step[(steps - 1) % nb])
+    e1.record(s_out)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / 1e3, h2d, d2h
 
@@ -529,7 +552,7 @@ def run_ours(args):
     by = algorithmic_bytes(p)
 
     e2e_steps = max(3, min(args.steps, 2000))
-    e2e_t, h2d, d2h = e2e_measure(p, sets[0], e2e_steps, 3, stream)
+    e2e_t, h2d, d2h = e2e_measure(p, sets, e2e_steps, 3, stream)
     e2e_t = max_over_ranks(e2e_t, ws, dev)
     e2e_val = sum_over_ranks(p.T * e2e_steps, ws, dev) / e2e_t
 
