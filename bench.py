@@ -42,9 +42,18 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = [os.path.join(ROOT, "gather_matmul_b200", "csrc", f)
-                  for f in ("bgmv.cu", "bgmv_fused.cu", "group.cu", "sgmv_tc.cu", "common.cuh",
-                            "ptx.cuh")]
+# the source files each kernel is built from: a DRAM-traffic figure taken
+# with ncu stays valid until one of them changes
+_CSRC = os.path.join(ROOT, "gather_matmul_b200", "csrc")
+_COMMON = ("common.cuh", "ptx.cuh", "internal.h")
+KERNEL_SOURCES = {
+    "bgmv_fused_kernel": ("bgmv_fused.cu", "tmap.cu") + _COMMON,
+    "sgmv_shrink_tc_kernel": ("sgmv_tc.cu", "tmap.cu") + _COMMON,
+    "sgmv_expand_tc_kernel": ("sgmv_tc.cu", "tmap.cu") + _COMMON,
+    "shrink_items_kernel": ("bgmv.cu",) + _COMMON,
+    "expand_items_kernel": ("bgmv.cu",) + _COMMON,
+    "group_kernel": ("group.cu",) + _COMMON,
+}
 
 
 # --------------------------------------------------------------------------
@@ -94,11 +103,12 @@ def aggregate(values_per_rank_tokens, elapsed_max_s):
     return float(sum(values_per_rank_tokens)) / elapsed_max_s
 
 
-def kernel_source_hash():
+def kernel_source_hash(kernel):
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
-        if os.path.exists(f):
-            h.update(open(f, "rb").read())
+    for f in KERNEL_SOURCES[kernel]:
+        path = os.path.join(_CSRC, f)
+        if os.path.exists(path):
+            h.update(open(path, "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -122,14 +132,13 @@ def measured_bf16_tflops():
 
 def profile_traffic(kernel):
     """DRAM bytes per launch from the committed ncu summary, or None when it
-    is missing or was taken on other kernel sources."""
-    if not os.path.exists(PROFILE_TRAFFIC):
+    is missing or was taken on other sources of that kernel."""
+    if not os.path.exists(PROFILE_TRAFFIC) or kernel not in KERNEL_SOURCES:
         return None
-    d = json.load(open(PROFILE_TRAFFIC))
-    if d.get("source_hash") != kernel_source_hash():
+    k = json.load(open(PROFILE_TRAFFIC)).get("kernels", {}).get(kernel)
+    if k is None or k.get("source_hash") != kernel_source_hash(kernel):
         return None
-    k = d.get("kernels", {}).get(kernel)
-    return None if k is None else k.get("dram_bytes_per_launch")
+    return k.get("dram_bytes_per_launch")
 
 
 # --------------------------------------------------------------------------

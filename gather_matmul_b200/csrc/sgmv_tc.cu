@@ -362,6 +362,7 @@ constexpr int kMaxRuns = 64;
 constexpr int kMaxSegTC = 2048;          // longer segment lists use the item kernels
 constexpr int kMaxSegChunks = kMaxSegTC / 32 + 1;
 constexpr int kSwapMax = 64;             // tiles of at most this many rows swap operands
+constexpr int kSegCache = 256;           // segment lists up to this long are read once
 
 struct ExpandTCParams {
   CUtensorMap tmB[LORA_MAX_SLICES];      // B_i as [S*D_out_i rows, r cols], box {r, 128}
@@ -399,10 +400,14 @@ struct ExpandSmem {
   static constexpr size_t kOffTok = kOffInv + 2 * kTM * 4;            // int [2][128]
   static constexpr size_t kOffRun = kOffTok + 2 * kTM * 4;            // ExpRun [kMaxRuns]
   static constexpr size_t kOffChunk = kOffRun + kMaxRuns * sizeof(ExpRun);   // int64 [chunks]
-  static constexpr size_t kOffBar = kOffChunk + 8 * kMaxSegChunks;
+  static constexpr size_t kOffSeg = (kOffChunk + 8 * kMaxSegChunks + 15) & ~size_t(15);   // int4 [kSegCache]
+  static constexpr size_t kOffBar = kOffSeg + 16 * kSegCache;
   static constexpr int kNBar = 2 * kYS + 8;
   static constexpr size_t kOffMisc = kOffBar + 8 * kNBar;             // tmem, n_runs, next
   static constexpr size_t kTotal = kOffMisc + 64 + 1024;
+  static_assert(kOffB % 1024 == 0 && kOffHL % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+  static_assert(kOffInv % 16 == 0 && kOffTok % 16 == 0 && kOffRun % 8 == 0, "alignment");
+  static_assert(kOffChunk % 8 == 0 && kOffSeg % 16 == 0 && kOffBar % 8 == 0, "alignment");
 };
 
 // Bytes a pair moves, in units the schedule balances: the B tile, the valid
@@ -417,6 +422,16 @@ struct SegView {
   const int32_t* ss;
   const int32_t* sa;
   int n_seg, T, S, implicit_slots;
+  int4* cache;                           // shared-memory copy of the first kSegCache segments
+  // the same, from the copy when the whole list is in it
+  __device__ __forceinline__ void get_cached(int s, int& a, int& b, int& ad) const {
+    if (n_seg <= kSegCache) {
+      const int4 c = s < n_seg ? cache[s] : make_int4(0, 0, -1, 0);
+      a = c.x; b = c.y; ad = c.z;
+    } else {
+      get(s, a, b, ad);
+    }
+  }
   // segment s clamped into [0, T]; adapter -1 when it has none or is out of range
   __device__ __forceinline__ void get(int s, int& a, int& b, int& ad) const {
     a = 0; b = 0; ad = -1;
@@ -450,7 +465,9 @@ __device__ int64_t seg_chunk_weights(const SegView& sv, int64_t* chunkW) {
 #pragma unroll
     for (int u = 0; u < 4; ++u) {          // all loads first, then the reductions
       int a, b, ad;
-      sv.get((c0 + u) * 32 + lane, a, b, ad);
+      const int sidx = (c0 + u) * 32 + lane;
+      sv.get(sidx, a, b, ad);
+      if (sidx < kSegCache) sv.cache[sidx] = make_int4(a, b, ad, 0);
       w[u] = seg_weight<R>(a, b, ad);
     }
 #pragma unroll
@@ -495,7 +512,7 @@ __device__ int build_runs(const SegView& sv, const int64_t* chunkW, int64_t Wt,
         continue;
       }
       int a, b, ad;
-      sv.get(c * 32 + lane, a, b, ad);
+      sv.get_cached(c * 32 + lane, a, b, ad);
       const int64_t sw = nt * seg_weight<R>(a, b, ad);
       int64_t incl = sw;
 #pragma unroll
@@ -577,7 +594,8 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   int64_t* sRange = reinterpret_cast<int64_t*>(smem + L::kOffMisc + 8);   // lo, hi, Wt, next
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 48);
 
-  const SegView sv{P.seg_starts, P.seg_adapter, P.n_seg, P.T, P.S, P.implicit_slots};
+  const SegView sv{P.seg_starts, P.seg_adapter, P.n_seg, P.T, P.S, P.implicit_slots,
+                   reinterpret_cast<int4*>(smem + L::kOffSeg)};
   if (blockIdx.x == 0 && !P.implicit_slots)
     validate_segments(P.seg_starts, P.seg_adapter, P.n_seg, P.T, P.S, P.bad_index, P.bad_meta);
   int ntiles[LORA_MAX_SLICES];
@@ -651,11 +669,59 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
         const ExpRun rn = runs[ri];
         const int hb = ul & 1;
         if (ul >= 2) ok &= ptx::mbar_wait_ff(&hlempty[hb], ((ul >> 1) - 1) & 1, sAbort);
-        // operand rows: token, hi / lo after an exact power-of-two rescale
-        // 2^(7-e) (e = exponent of the row's max |buf|), and the inverse scale
+        // this thread's operand row: its token first (the gathers need every
+        // row's token), then the loads of the run's first pairs whose stages
+        // are free without waiting, then the hi / lo rows, so that the buf
+        // reads overlap those loads
+        const int m = lt;
+        const int tok = m < rn.valid ? (P.perm ? P.perm[rn.m0 + m] : rn.m0 + m) : -1;
+        sTok[hb * kTM + m] = tok;
+        asm volatile("bar.sync 4, 128;" ::: "memory");   // every row's token is known
+        const int* toks = sTok + hb * kTM;
+        const int Dout = P.D_out[rn.slice];
+        const int64_t ycol0 = P.y_col_off[rn.slice];
+        const bool tiled = P.perm == nullptr && rn.valid == kTM;
+        const int ngroups = (rn.valid + 3) / 4;
+        int my_ops = 0;
+        if (!tiled)
+          for (int o = pw; o < 2 * ngroups; o += 4) ++my_ops;
+        auto issue_pair = [&](int j, int pq) {
+          const int s = pq % kYS;
+          if (pq >= kYS) ok &= ptx::mbar_wait_ff(&empty[s], ((pq / kYS) - 1) & 1, sAbort);
+          const int n0 = j * kNT;
+          char* ys = sY + (size_t)s * L::kYBytes;
+          const uint32_t bytes =
+              (uint32_t)(my_ops * 512) +
+              (pw == 0 ? (uint32_t)L::kBBytes + (tiled ? (uint32_t)L::kYBytes : 0u) : 0u);
+          if (lane == 0) {
+            ptx::mbar_arrive_expect_tx(&full[s], bytes);
+            if (pw == 0) {
+              ptx::tma_load_2d(sB + (size_t)s * L::kBBytes, &P.tmB[rn.slice], 0,
+                               rn.adapter * Dout + n0, &full[s]);
+              if (tiled) {
+                ptx::tma_load_2d(ys, &P.tmY, (int)(ycol0 + n0), rn.m0, &full[s]);
+                ptx::tma_load_2d(ys + L::kYHalf, &P.tmY, (int)(ycol0 + n0 + 64), rn.m0, &full[s]);
+              }
+            }
+          }
+          __syncwarp();
+          if (!tiled) {
+            // 2 halves x ngroups 4-row gathers: op o -> warp o % 4, lane o / 4
+            for (int o = pw + 4 * lane; o < 2 * ngroups; o += 128) {
+              const int g = o >> 1, h = o & 1;
+              int rr[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) rr[q] = toks[4 * g + q < rn.valid ? 4 * g + q : 4 * g];
+              ptx::tma_gather4(ys + h * L::kYHalf + g * 512, &P.tmYg, (int)(ycol0 + n0 + 64 * h),
+                               rr[0], rr[1], rr[2], rr[3], &full[s]);
+            }
+          }
+        };
+        int j = rn.j0;
+        for (; j < rn.j1 && pl < kYS; ++j, ++pl) issue_pair(j, pl);
+        // hi / lo after an exact power-of-two rescale 2^(7-e) (e = exponent of
+        // the row's max |buf|), and the inverse scale
         {
-          const int m = lt;
-          const int tok = m < rn.valid ? (P.perm ? P.perm[rn.m0 + m] : rn.m0 + m) : -1;
           const float4* brow = reinterpret_cast<const float4*>(
               P.buf + (size_t)rn.slice * P.buf_slice_stride + (size_t)(tok < 0 ? 0 : tok) * R);
           float4 f[R / 4];
@@ -687,51 +753,11 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
             *reinterpret_cast<uint4*>(loP + off) = *reinterpret_cast<const uint4*>(l8);
           }
           sInv[hb * kTM + m] = __int_as_float((127 + e - 7) << 23);
-          sTok[hb * kTM + m] = tok;
           ptx::fence_proxy_async_smem();   // generic writes -> tensor-core operand reads
         }
-        asm volatile("bar.sync 4, 128;" ::: "memory");   // every row's token is known
-        if (lane == 0) ptx::mbar_arrive(&hlfull[hb]);
-        const int* toks = sTok + hb * kTM;
-        const int Dout = P.D_out[rn.slice];
-        const int64_t ycol0 = P.y_col_off[rn.slice];
-        const bool tiled = P.perm == nullptr && rn.valid == kTM;
-        const int ngroups = (rn.valid + 3) / 4;
-        int my_ops = 0;
-        if (!tiled)
-          for (int o = pw; o < 2 * ngroups; o += 4) ++my_ops;
-        for (int j = rn.j0; j < rn.j1; ++j, ++pl) {
-          const int s = pl % kYS;
-          if (pl >= kYS) ok &= ptx::mbar_wait_ff(&empty[s], ((pl / kYS) - 1) & 1, sAbort);
-          const int n0 = j * kNT;
-          char* ys = sY + (size_t)s * L::kYBytes;
-          const uint32_t bytes =
-              (uint32_t)(my_ops * 512) +
-              (pw == 0 ? (uint32_t)L::kBBytes + (tiled ? (uint32_t)L::kYBytes : 0u) : 0u);
-          if (lane == 0) {
-            ptx::mbar_arrive_expect_tx(&full[s], bytes);
-            if (pw == 0) {
-              ptx::tma_load_2d(sB + (size_t)s * L::kBBytes, &P.tmB[rn.slice], 0,
-                               rn.adapter * Dout + n0, &full[s]);
-              if (tiled) {
-                ptx::tma_load_2d(ys, &P.tmY, (int)(ycol0 + n0), rn.m0, &full[s]);
-                ptx::tma_load_2d(ys + L::kYHalf, &P.tmY, (int)(ycol0 + n0 + 64), rn.m0, &full[s]);
-              }
-            }
-          }
-          __syncwarp();
-          if (!tiled) {
-            // 2 halves x ngroups 4-row gathers: op o -> warp o % 4, lane o / 4
-            for (int o = pw + 4 * lane; o < 2 * ngroups; o += 128) {
-              const int g = o >> 1, h = o & 1;
-              int rr[4];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) rr[q] = toks[4 * g + q < rn.valid ? 4 * g + q : 4 * g];
-              ptx::tma_gather4(ys + h * L::kYHalf + g * 512, &P.tmYg, (int)(ycol0 + n0 + 64 * h),
-                               rr[0], rr[1], rr[2], rr[3], &full[s]);
-            }
-          }
-        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&hlfull[hb]);   // one arrival per load warp
+        for (; j < rn.j1; ++j, ++pl) issue_pair(j, pl);
       }
     } else if (warp == kExpMma) {
       // ---------------- MMA issue
@@ -998,11 +1024,12 @@ cudaError_t shrink_tc_launch(const ShrinkArgs& a, const SegArgs& sg, lora_dtype 
   P.bad_meta = const_cast<int*>(&hdr->bad_meta);
   const int max_tiles = (a.T + kTM - 1) / kTM + sg.n_seg;
   const int nkb_all = (a.D + kBK - 1) / kBK;
-  // split K across a cluster when there are too few tiles to fill the GPU:
-  // up to 16 ranks (a non-portable cluster size, used when the device takes it)
+  // split K across a cluster when there are too few tiles for about 1.5 CTAs
+  // per SM, each rank keeping at least 8 K blocks: up to 16 ranks (a
+  // non-portable cluster size, used when the device takes it)
   const int nsm = sm_count();
   int KS = 1;
-  while (KS < 16 && (long)max_tiles * a.n_slices * KS < nsm && nkb_all >= 4 * KS) KS *= 2;
+  while (KS < 16 && 2L * max_tiles * a.n_slices * KS < 3L * nsm && nkb_all >= 16 * KS) KS *= 2;
   auto kern = sgmv_shrink_tc_kernel<E, R>;
   const size_t smem = ShrinkSmem<R>::kTotal;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -56,15 +56,19 @@ def test_rotation_sets_cover_three_l2():
 
 
 def test_profile_traffic_requires_matching_sources(tmp_path, monkeypatch):
+    import json
     f = tmp_path / "traffic.json"
     monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(f))
-    assert bench.profile_traffic("bgmv_fused_kernel") is None
-    import json
-    f.write_text(json.dumps({"source_hash": "stale", "kernels": {"k": {"dram_bytes_per_launch": 5}}}))
-    assert bench.profile_traffic("k") is None
-    f.write_text(json.dumps({"source_hash": bench.kernel_source_hash(),
-                             "kernels": {"k": {"dram_bytes_per_launch": 5}}}))
-    assert bench.profile_traffic("k") == 5
+    k = "bgmv_fused_kernel"
+    assert bench.profile_traffic(k) is None
+    f.write_text(json.dumps({"kernels": {k: {"source_hash": "stale", "dram_bytes_per_launch": 5}}}))
+    assert bench.profile_traffic(k) is None
+    f.write_text(json.dumps({"kernels": {k: {"source_hash": bench.kernel_source_hash(k),
+                                             "dram_bytes_per_launch": 5}}}))
+    assert bench.profile_traffic(k) == 5
+    assert bench.profile_traffic("not_a_kernel") is None
+    # each kernel's figure follows its own sources only
+    assert bench.kernel_source_hash(k) != bench.kernel_source_hash("sgmv_expand_tc_kernel")
 
 
 def _free_port():
