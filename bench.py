@@ -601,6 +601,7 @@ def run_ours(args):
 def detail_all(args, stream, peak, peak_kind):
     """Per-projection numbers of every workload (not the headline line)."""
     out = {}
+    layer = []
     tf_peak = measured_bf16_tflops()
     for n in (1, 2, 3, 4, 5):
         for p in W.config(n):
@@ -629,11 +630,36 @@ def detail_all(args, stream, peak, peak_kind):
                 "tensor_frac_step": round(fl / t / 1e12 / tf_peak, 4),
                 "roofline_frac_step": round(max(fl / (tf_peak * 1e12), by["step"] / (peak * 1e9))
                                             / t, 4),
+                "frac_step_vs_8tbs": round(by["step"] / t / 8e12, 4),
                 "bytes": by,
             }
+            if n == 3:
+                layer.append((t, by["step"], p.T))
             del sets
             torch.cuda.empty_cache()
+    # the three fused-slice projections of one decoder layer, back to back
+    t3 = sum(v[0] for v in layer)
+    b3 = sum(v[1] for v in layer)
+    out["cfg3:layer_sum"] = {"us_per_layer": round(t3 * 1e6, 3),
+                             "tokens_per_s": round(layer[0][2] / t3, 1),
+                             "gbs": round(b3 / t3 / 1e9, 1), "frac": round(b3 / t3 / 1e9 / peak, 4)}
+    out["idle_call_us"] = idle_call_us()
     return out
+
+
+def idle_call_us(calls=2000):
+    """Host time of a per-token call when no token has an adapter (has_active
+    = 0): the library returns before any launch, so this is the whole cost of
+    LoRA being enabled but idle."""
+    from gather_matmul_b200 import ops
+    p = W.config(2)[0]
+    d = DeviceSet(p)
+    for _ in range(10):
+        ops.bgmv(d.x, d.A, d.B, d.idx, d.y, d.buf, d.meta, p.scale, has_active=False)
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        ops.bgmv(d.x, d.A, d.B, d.idx, d.y, d.buf, d.meta, p.scale, has_active=False)
+    return round((time.perf_counter() - t0) / calls * 1e6, 3)
 
 
 # --------------------------------------------------------------------------
