@@ -650,16 +650,35 @@ def detail_all(args, stream, peak, peak_kind):
 def idle_call_us(calls=2000):
     """Host time of a per-token call when no token has an adapter (has_active
     = 0): the library returns before any launch, so this is the whole cost of
-    LoRA being enabled but idle."""
-    from gather_matmul_b200 import ops
+    LoRA being enabled but idle.  Through the Python binding, and through the
+    C ABI with the arguments marshalled once."""
+    import ctypes
+    from gather_matmul_b200 import _lib, ops
     p = W.config(2)[0]
     d = DeviceSet(p)
+    out = {}
     for _ in range(10):
         ops.bgmv(d.x, d.A, d.B, d.idx, d.y, d.buf, d.meta, p.scale, has_active=False)
     t0 = time.perf_counter()
     for _ in range(calls):
         ops.bgmv(d.x, d.A, d.B, d.idx, d.y, d.buf, d.meta, p.scale, has_active=False)
-    return round((time.perf_counter() - t0) / calls * 1e6, 3)
+    out["python_op"] = round((time.perf_counter() - t0) / calls * 1e6, 3)
+    vp = ctypes.c_void_p
+    ptrs = lambda ts: (vp * len(ts))(*[t.data_ptr() for t in ts])
+    n = len(d.B)
+    args = (_lib.LORA_F16 if p.dtype == W.F16 else _lib.LORA_BF16, p.T, p.D, p.r, p.S, n,
+            vp(d.x.data_ptr()), p.D, ptrs(d.A), 0, ptrs(d.B),
+            (ctypes.c_int32 * n)(*[b.shape[1] for b in d.B]), ctypes.c_float(p.scale),
+            vp(d.y.data_ptr()), d.y.stride(0), (ctypes.c_int64 * n)(*[int(o) for o in p.col_off]),
+            vp(d.buf.data_ptr()), vp(d.idx.data_ptr()), 0, 0, vp(d.meta.data_ptr()),
+            d.meta.numel(), vp(torch.cuda.current_stream().cuda_stream))
+    fn = _lib.load().lora_bgmv
+    assert fn(*args) == 0
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        fn(*args)
+    out["c_abi"] = round((time.perf_counter() - t0) / calls * 1e6, 3)
+    return out
 
 
 # --------------------------------------------------------------------------
