@@ -124,3 +124,45 @@ def test_sgmv_many_mixed_segments():
     p = W.make_problem("mixed_segments", W.BF16, T=int(ss[-1]), D=1024, r=32, S=6,
                        d_out=[512], scale=0.5, seed=13, segments=(ss, sa))
     _run_and_check(p)
+
+
+RANDOM_SEGMENT_SEEDS = list(range(8))
+
+
+@pytest.mark.parametrize("seed", RANDOM_SEGMENT_SEEDS)
+def test_sgmv_random_segment_layouts(seed):
+    """Random segment lists (empty segments, repeats, no-adapter runs, lengths
+    around the 64- and 128-row tile boundaries) over 1-3 slices whose widths
+    are not multiples of 128: every tile shape and schedule split of the
+    tensor-core kernels against the oracle."""
+    rng = np.random.default_rng(100 + seed)
+    n_seg = int(rng.integers(1, 60))
+    lens = rng.choice([0, 1, 3, 8, 31, 63, 64, 65, 127, 128, 129, 200, 257], size=n_seg)
+    if lens.sum() == 0:
+        lens[0] = 5
+    ss = np.concatenate([[0], np.cumsum(lens)])
+    S = int(rng.integers(1, 9))
+    sa = rng.integers(-1, S, size=n_seg)
+    r = int(rng.choice([16, 32, 64]))
+    d_out = [int(rng.choice([8, 136, 256, 392])) for _ in range(int(rng.integers(1, 4)))]
+    dt = W.BF16 if seed % 2 else W.F16
+    p = W.make_problem("random_segments", dt, T=int(ss[-1]), D=int(rng.choice([64, 264, 1024])),
+                       r=r, S=S, d_out=d_out, scale=0.75, seed=200 + seed, segments=(ss, sa))
+    _run_and_check(p)
+
+
+@pytest.mark.parametrize("seed", list(range(6)))
+def test_grouped_random_batches(seed):
+    """Random per-token batches with at least 16 tokens per slot on average,
+    so the grouping feeds the tensor-core kernels: skewed and uniform slot
+    popularity, tokens without an adapter, slot groups of every size."""
+    rng = np.random.default_rng(300 + seed)
+    S = int(rng.integers(1, 24))
+    T = int(16 * S + rng.integers(0, 700))
+    kind = ["uniform", "uniform_neg", "zipf", "frac_neg", "single", "uniform"][seed]
+    r = [16, 32, 64][seed % 3]
+    d_out = [int(rng.choice([64, 200, 512])) for _ in range(1 + seed % 3)]
+    p = W.make_problem("grouped_random", W.BF16 if seed % 2 else W.F16, T=T,
+                       D=int(rng.choice([128, 776, 2048])), r=r, S=S, d_out=d_out, scale=1.25,
+                       seed=400 + seed, idx_kind=kind, frac_neg=0.2)
+    _run_and_check(p)
