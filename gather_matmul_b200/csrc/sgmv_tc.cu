@@ -815,6 +815,10 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
         const bool tiled = P.perm == nullptr && rn.valid == kTM;
         for (int j = rn.j0; j < rn.j1; ++j, ++pl) {
           const int s = pl % kYS, a = pl & 1;
+          // a swapped pair is handled by one group of four warps (one per TMEM
+          // lane quadrant), the group of its accumulator: consecutive small
+          // pairs overlap; a full pair by all eight
+          if (swap && a != h) continue;
           const int n0 = j * kNT, nn = min(kNT, Dout - n0);
           ok &= ptx::mbar_wait_ff(&accfull[a], (pl >> 1) & 1, sAbort);
           ok &= ptx::mbar_wait_ff(&full[s], (pl / kYS) & 1, sAbort);
@@ -899,13 +903,12 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
               ptx::fence_proxy_async_smem();
             }
           } else {
-            // swapped: thread = output column 32q + lane; groups of 8 tokens
-            // alternate between the two warps of the quadrant
+            // swapped: thread = output column 32q + lane, all groups of 8 tokens
             const int col = q * 32 + lane;
             const int hc = col >> 6, cc = col & 63;
             char* cbase = ys + hc * L::kYHalf + (cc & 7) * 2;
             const int ng = (rn.valid + 7) / 8;
-            for (int g = h; g < ng; g += 2) {
+            for (int g = 0; g < ng; ++g) {
               uint32_t r[8];
               ptx::tc_ld8(tacc + 8 * g, r);
               const float4 i0 = *reinterpret_cast<const float4*>(invs + 8 * g);
@@ -929,21 +932,22 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
             }
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&accempty[a]);
-            asm volatile("bar.sync 3, 256;" ::: "memory");   // every column of every row done
+            if (lane == 0) ptx::mbar_arrive_cnt(&accempty[a], 2);   // four warps count as eight
+            asm volatile("bar.sync %0, 128;" ::"r"(1 + h) : "memory");   // the group's columns done
             // rows 0 .. valid-1, 16 chunks each: e -> (row e / 16, chunk e % 16);
-            // at most 64 rows: four pieces per thread, all read before any store
-            uint4 v[4];
+            // at most 64 rows: eight pieces per thread, all read before any store
+            const int gl = q * 32 + lane;
+            uint4 v[8];
 #pragma unroll
-            for (int it = 0; it < 4; ++it) {
-              const int e = warp * 32 + lane + 256 * it;
+            for (int it = 0; it < 8; ++it) {
+              const int e = gl + 128 * it;
               const int mr = min(e >> 4, kSwapMax - 1), hh = (e >> 3) & 1, ch = e & 7;
               v[it] = *reinterpret_cast<const uint4*>(ys + hh * L::kYHalf + mr * 128 +
                                                       ((ch ^ (mr & 7)) << 4));
             }
 #pragma unroll
-            for (int it = 0; it < 4; ++it) {
-              const int e = warp * 32 + lane + 256 * it;
+            for (int it = 0; it < 8; ++it) {
+              const int e = gl + 128 * it;
               const int mr = e >> 4, hh = (e >> 3) & 1, ch = e & 7;
               if (mr < rn.valid && 64 * hh + 8 * ch < nn)
                 *reinterpret_cast<uint4*>(ycol + (size_t)toks[mr] * P.ldy + n0 + 64 * hh + 8 * ch) =
@@ -952,7 +956,7 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
             ptx::fence_proxy_async_smem();
           }
           __syncwarp();
-          if (lane == 0 && deferred != s) ptx::mbar_arrive(&empty[s]);
+          if (lane == 0 && deferred != s) ptx::mbar_arrive_cnt(&empty[s], swap ? 2u : 1u);
         }
         // done with this run's tokens and scales
         __syncwarp();
