@@ -128,6 +128,9 @@ LORA_API lora_status lora_group(int T, int S, const int32_t* idx, void* meta, si
  *               untouched (pull 25914: no LoRA kernels, no zeroing).
  *   meta        the workspace lora_group filled from this batch's idx on this
  *               stream (or one ordered before it).
+ * With r >= 16 and T >= 16 * S the slot groups of the grouping run on tcgen05
+ * tensor cores (x rows gathered through the grouping permutation); otherwise
+ * on CUDA cores.
  */
 LORA_API lora_status lora_shrink(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
                         const void* x, int64_t ldx, const void* const* A, float* buf,
@@ -152,6 +155,7 @@ LORA_API lora_status lora_shrink(lora_dtype dtype, int T, int D, int r, int S, i
  *   y_col_off         host int64 [n_slices], first column of each slice in y;
  *                     slices must not overlap.
  *   has_active, meta  as for lora_shrink.
+ * Tensor cores or CUDA cores as for lora_shrink.
  */
 LORA_API lora_status lora_expand(lora_dtype dtype, int T, int r, int S, int n_slices,
                         const float* buf, int64_t buf_slice_stride, const void* const* B,
@@ -210,7 +214,7 @@ LORA_API int lora_bgmv_launches(lora_dtype dtype, int T, int D, int r, int S, in
  * Malformed segments are counted as bad (LORA_ERR_BAD_INDEX from
  * lora_check_errors); the rows they would cover are then unspecified, but no
  * access leaves the buffers.  Runs on tcgen05 tensor cores when r >= 16 and
- * dtype is bf16 or fp16, else on CUDA cores.
+ * n_seg <= 2048, else on CUDA cores.
  */
 LORA_API lora_status lora_shrink_segment(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
                                 const void* x, int64_t ldx, const void* const* A,
