@@ -48,7 +48,9 @@ namespace {
 constexpr int kTM = 128;          // token rows per tile (MMA M)
 constexpr int kBK = 64;           // K elements per pipeline stage: one 128-byte row
 template <int R>
-constexpr int stages_for() { return R <= 32 ? 6 : 4; }   // two CTAs per SM at every rank
+// stages of 16 KB x + r x 128 B adapter: 108 / 100 / 96 KB for r = 16 / 32 / 64,
+// so that two CTAs fit per SM at every rank
+constexpr int stages_for() { return R == 16 ? 6 : (R == 32 ? 5 : 4); }
 constexpr int kNT = 128;          // expand output columns per CTA (MMA N)
 
 struct TileInfo {
@@ -155,6 +157,11 @@ struct ShrinkSmem {
   static constexpr size_t kBar = (size_t)kStageBytes * kStages;
   static constexpr size_t kTotal = kBar + 8 * (2 * kStages + 1) + 64 + 1024;
 };
+
+static_assert(2 * (ShrinkSmem<16>::kTotal + 1024) <= 228 * 1024 &&
+                  2 * (ShrinkSmem<32>::kTotal + 1024) <= 228 * 1024 &&
+                  2 * (ShrinkSmem<64>::kTotal + 1024) <= 228 * 1024,
+              "two shrink CTAs per SM");
 
 // warps 0-3: loads (one per SM sub-partition, so small gathers issue four-wide),
 // then the epilogue on TMEM lane quadrant = warp; warp 4: MMA issue.
