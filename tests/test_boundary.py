@@ -211,3 +211,36 @@ def test_stream_and_graph_capture():
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(d.y, y_eager)
+
+
+@pytest.mark.parametrize("path", ["grouped", "fused", "segments"])
+def test_power_of_two_scale_scales_y_exactly(path):
+    # With y_old = 0, y = rn(scale * acc): a power-of-two scale commutes with
+    # the rounding, so scale 4 gives exactly 4x the scale-1 result, element for
+    # element (no value here comes near the fp16/bf16 range limits).
+    if path == "segments":
+        ss, sa = np.array([0, 64, 200, 330]), np.array([1, -1, 0])
+        p = W.make_problem("s", W.BF16, T=330, D=1024, r=32, S=2, d_out=[384], scale=1.0,
+                           seed=21, segments=(ss, sa))
+    else:
+        # bf16: fp32's exponent range, so no result is subnormal (in fp16 a
+        # subnormal would round at a fixed absolute step and break the identity)
+        p = W.make_problem("s", W.BF16, T=256, D=1024, r=16, S=4, d_out=[512], scale=1.0, seed=22,
+                           idx_kind="uniform_neg")
+    ys = []
+    for scale in (1.0, 4.0):
+        d = Dev(p)
+        d.y.zero_()
+        if path == "fused":
+            ops.bgmv(d.x, d.A, d.B, d.idx, d.y, d.buf, d.meta, scale, y_col_off=p.col_off)
+        else:
+            d.shrink()
+            b = d.buf
+            if p.segmented:
+                ops.expand_segment(b, d.B, d.ss, d.sa, d.y, d.meta, scale, y_col_off=p.col_off)
+            else:
+                ops.expand(b, d.B, d.y, d.meta, scale, y_col_off=p.col_off)
+        torch.cuda.synchronize()
+        ys.append(oracle.decode(p.dtype, host_bits(d.y)))
+    assert np.any(ys[0] != 0)
+    assert np.array_equal(ys[1], 4.0 * ys[0])
