@@ -2,19 +2,28 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
 
-One step = one pass of the whole per-token (BGMV) path over one batch:
-group-by-slot metadata, shrink into the fp32 intermediate, expand into the
-output slices.  At N=1 the workload is the decode batch at a Llama-3-8B
-q_proj shape (T=256 tokens, D=D_out=4096, 32 slots, rank 16, fp16, scale 2),
-unless --config picks another.  Inputs are seeded synthetic tensors of that
-shape; adapter weights are random, not trained.
+One step = one pass of the whole path over one batch: for a per-token (BGMV)
+batch the public one-call entry point (group-by-slot, shrink into the fp32
+intermediate, expand into the output slices); for a segment (SGMV) batch the
+segment shrink and expand.  At N=1 the headline workload is the largest
+single-GPU one, the large mixed batch (T=4096 single tokens, D=D_out=8192,
+128 slots, rank 32, Zipf(1.1) adapter popularity with 10 % of tokens on the
+base model only, unsorted, bf16), unless --config picks another.  Inputs are
+seeded synthetic tensors of that shape; adapter weights are random, not
+trained.
 
-Timing: K steps are captured in CUDA graphs and replayed, each step on the
-next of several input sets whose total size is more than three times the L2
-cache, so every step reads cold HBM.  CUDA events on the launching stream,
-barrier + synchronize on both sides, max over ranks.  Multi-GPU runs are
-independent data-parallel replicas (each rank its own token batch, adapters
-replicated; no collective on the data path): weak scaling.
+Timing: the K steps are captured in CUDA graphs, replayed once untimed (with
+the warm-up steps) and then timed; each step runs on the next of several
+input sets whose total size is more than three times the L2 cache, so every
+step reads cold HBM.  CUDA events on the launching stream, barrier +
+synchronize on both sides, max over ranks.  Every kernel's own time comes from
+a separate graph of at least 256 launches, also replayed once before timing.
+The end-to-end figure times at least 100 ms of steps through the public call
+with the inputs copied from pinned host memory and the result read back.
+The line carries a per-workload block ("configs") with every workload's step
+and kernel times and their fractions of the HBM and tensor rooflines.
+Multi-GPU runs are independent data-parallel replicas (each rank its own token
+batch, adapters replicated; no collective on the data path): weak scaling.
 
 Rank 0 prints one JSON line.  --impl reference times the CPU oracle (the
 plain fp64 definition) on bounded samples of the same workload instead.
@@ -23,6 +32,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -53,6 +63,7 @@ KERNEL_SOURCES = {
     "shrink_items_kernel": ("bgmv.cu",) + _COMMON,
     "expand_items_kernel": ("bgmv.cu",) + _COMMON,
     "group_kernel": ("group.cu",) + _COMMON,
+    "segment_items_kernel": ("group.cu",) + _COMMON,
 }
 
 
@@ -130,13 +141,16 @@ def measured_bf16_tflops():
     return FALLBACK_BF16_TFLOPS
 
 
-def profile_traffic(kernel):
+def profile_traffic(kernel, workload=None):
     """DRAM bytes per launch from the committed ncu summary, or None when it
-    is missing or was taken on other sources of that kernel."""
+    is missing, was taken on another workload, or on other sources of that
+    kernel."""
     if not os.path.exists(PROFILE_TRAFFIC) or kernel not in KERNEL_SOURCES:
         return None
     k = json.load(open(PROFILE_TRAFFIC)).get("kernels", {}).get(kernel)
     if k is None or k.get("source_hash") != kernel_source_hash(kernel):
+        return None
+    if workload is not None and k.get("workload") != workload:
         return None
     return k.get("dram_bytes_per_launch")
 
@@ -240,6 +254,56 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------
+# which kernels each call launches (mirrors the library's dispatch rules)
+# --------------------------------------------------------------------------
+def grouped_tc(p):
+    """Per-token batches with r >= 16 and at least 16 tokens per slot on
+    average run their slot groups through the tensor-core kernels."""
+    return p.r >= 16 and p.T >= 16 * p.S and p.D % 8 == 0
+
+
+def kernels_of(p, what, fused_fits):
+    """Kernel names behind one timed call of a step."""
+    if what == "fused":
+        return ["bgmv_fused_kernel"]
+    if what == "group":
+        return ["group_kernel"]
+    if p.segmented:
+        if p.r >= 16 and len(p.seg_adapter) <= 2048:
+            return ["sgmv_%s_tc_kernel" % what]
+        return ["segment_items_kernel", "%s_items_kernel" % what]
+    return ["sgmv_%s_tc_kernel" % what] if grouped_tc(p) else ["%s_items_kernel" % what]
+
+
+def kernel_calls(p, fused_fits):
+    """The separately timed calls that make one step."""
+    if p.segmented:
+        return ["shrink", "expand"]
+    return ["fused"] if fused_fits else ["group", "shrink", "expand"]
+
+
+def call_bytes(p, what):
+    by = algorithmic_bytes(p)
+    if what == "fused":
+        return by["shrink"] + by["expand"]
+    return by[what]
+
+
+def call_flops(p, what):
+    Ta, _ = active_stats(p)
+    sh = 2 * Ta * p.r * p.D * len(p.A)
+    ex = 2 * Ta * p.r * sum(p.d_out)
+    return {"fused": sh + ex, "shrink": sh, "expand": ex, "group": 0}[what]
+
+
+def e2e_steps_for(step_s, steps, min_s=0.1, cap=20000):
+    """Steps of the end-to-end loop: at least `steps`, and enough for
+    min_s seconds at the estimated time per step."""
+    need = math.ceil(round(min_s / max(step_s, 1e-9), 6))
+    return int(max(steps, min(cap, need)))
+
+
+# --------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------
 class DeviceSet:
@@ -279,14 +343,8 @@ def fused(p):
                                                    p.d_out) == 1
 
 
-def kernel_list(p):
-    if p.segmented:
-        return ["shrink", "expand"]
-    return ["fused"] if fused(p) else ["group", "shrink", "expand"]
-
-
 def step_calls(p, d, what="step"):
-    """Enqueue one step (or one kernel of it) on the current stream."""
+    """Enqueue one step (or one call of it) on the current stream."""
     from gather_matmul_b200 import ops
     shared = p.shared_A and p.n_slices > 1
     buf = d.buf[0] if shared else d.buf
@@ -297,26 +355,20 @@ def step_calls(p, d, what="step"):
             ops.expand_segment(buf, d.B, d.ss, d.sa, d.y, d.meta, p.scale, y_col_off=p.col_off)
         return
     if what in ("step", "fused"):
-        # the whole per-token path in one call (one launch when it fits), in
-        # plain stream order (no early start of the next launch)
+        # the public one-call per-token path: one fused launch when the shape
+        # fits, else group + shrink + expand; plain stream order
         ops.bgmv(d.x, d.A, d.B, d.idx, d.y, d.buf, d.meta, p.scale, y_col_off=p.col_off)
         return
     if what == "group":
         ops.group(d.idx, p.S, d.meta)
     if what == "shrink":
-        ops.shrink(d.x, d.A, d.buf, d.meta)
+        ops.shrink(d.x, d.A, d.idx, d.buf, d.meta)
     if what == "expand":
-        ops.expand(buf, d.B, d.y, d.meta, p.scale, y_col_off=p.col_off)
-
-
-def launches_per(p, what="step"):
-    if what != "step":
-        return 1
-    return 2 if p.segmented else (1 if fused(p) else 3)
+        ops.expand(buf, d.B, d.idx, d.y, d.meta, p.scale, y_col_off=p.col_off)
 
 
 class GraphRunner:
-    """K calls over rotating sets, as replays of captured CUDA graphs of up to
+    """Calls over rotating sets, as replays of captured CUDA graphs of up to
     G calls each."""
 
     def __init__(self, p, sets, stream, what="step", G=64):
@@ -345,29 +397,69 @@ class GraphRunner:
             plan.append(self._graph(rem, pos))
         return plan
 
-    @staticmethod
-    def run(plan):
-        for g in plan:
-            g.replay()
+    def run(self, plan):
+        with torch.cuda.stream(self.stream):
+            for g in plan:
+                g.replay()
 
 
-def time_plan(plan, stream):
+def time_plan(runner, plan):
+    """Device time of one replay of `plan`, measured with CUDA events on the
+    launching stream, synchronized on both sides."""
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    e0.record(stream)
-    with torch.cuda.stream(stream):
-        GraphRunner.run(plan)
-    e1.record(stream)
+    e0.record(runner.stream)
+    runner.run(plan)
+    e1.record(runner.stream)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / 1e3
 
 
-def make_sets(p, extra_copies):
+def warm_then_time(runner, K, warm_calls=0):
+    """Capture K calls, replay that exact plan untimed (at least once, and for
+    at least warm_calls calls), then time one replay of it."""
+    plan = runner.prepare(K)
+    for _ in range(max(1, -(-warm_calls // max(K, 1)))):
+        runner.run(plan)
+    torch.cuda.synchronize()
+    return time_plan(runner, plan)
+
+
+def make_sets(p):
     base = DeviceSet(p)
     n = rotation_sets(base.nbytes())
-    sets = [base] + [DeviceSet(p, src=base) for _ in range(n - 1)] if extra_copies else [base]
-    return sets
+    return [base] + [DeviceSet(p, src=base) for _ in range(n - 1)]
+
+
+def launches_per_step(p, d, stream):
+    """Kernels one step launches, counted by the library while one step is
+    recorded into a (discarded) graph."""
+    from gather_matmul_b200 import ops
+    g = torch.cuda.CUDAGraph()
+    torch.cuda.synchronize()
+    before = ops.launch_count()
+    with torch.cuda.graph(g, stream=stream):
+        step_calls(p, d, "step")
+    n = ops.launch_count() - before
+    del g
+    return n
+
+
+def kernel_times(p, sets, stream, reps, fused_fits):
+    """Average device time of each call of the step, from graphs of `reps`
+    calls each replayed once before timing."""
+    out = {}
+    if not p.segmented and not fused_fits:
+        # the grouping must exist on each set before its shrink / expand
+        with torch.cuda.stream(stream):
+            for d in sets:
+                step_calls(p, d, "group")
+        torch.cuda.synchronize()
+    for what in kernel_calls(p, fused_fits):
+        r = GraphRunner(p, sets, stream, what)
+        out[what] = warm_then_time(r, reps) / reps
+    return out
 
 
 def e2e_measure(p, dsets, steps, warmup, stream):
@@ -378,7 +470,8 @@ def e2e_measure(p, dsets, steps, warmup, stream):
     PCIe as one copy.  Steps are double-buffered over two device sets and
     three streams (copy in, compute, copy out), as a serving loop would
     overlap one batch's transfers with another's compute; every step still
-    moves all of its bytes."""
+    moves all of its bytes.  The loop runs at least `steps` steps and at least
+    100 ms."""
     import types
     nb = min(2, len(dsets))
     d0 = dsets[0]
@@ -424,17 +517,23 @@ def e2e_measure(p, dsets, steps, warmup, stream):
             done_out[i].record(s_out)
         used[i] = True
 
+    def timed(n):
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s_in)
+        for k in range(n):
+            one(k)
+        s_in.wait_stream(s_out)
+        e1.record(s_in)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 1e3
+
     for k in range(warmup):
         one(k)
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
-    for k in range(steps):
-        one(k)
-    e1.record(s_out)
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / 1e3, h2d, d2h
+    est = timed(max(warmup, 3)) / max(warmup, 3)
+    n = e2e_steps_for(est, steps)
+    return timed(n), n, h2d, d2h
 
 
 def cpu_baseline(p, budget_s=10.0):
@@ -471,56 +570,15 @@ def cpu_baseline(p, budget_s=10.0):
                       f"({el:.1f} s, fp64, OpenMP over tokens)"}
 
 
-def measure_config(p, steps, warmup, stream, detail=False):
-    sets = make_sets(p, extra_copies=True)
-    runner = GraphRunner(p, sets, stream, "step")
-    plan_w = runner.prepare(max(warmup, 1))
-    with torch.cuda.stream(stream):
-        GraphRunner.run(plan_w)
-    torch.cuda.synchronize()
-    plan = runner.prepare(steps)
-    return sets, runner, plan
-
-
-def kernel_times(p, sets, stream, reps):
-    out = {}
-    if not p.segmented and not fused(p):
-        # the group kernel must have run on each set before shrink / expand
-        for d in sets:
-            with torch.cuda.stream(stream):
-                step_calls(p, d, "group")
-        torch.cuda.synchronize()
-    for what in kernel_list(p):
-        r = GraphRunner(p, sets, stream, what)
-        plan = r.prepare(reps)
-        with torch.cuda.stream(stream):
-            GraphRunner.run(r.prepare(min(reps, 64)))
-        torch.cuda.synchronize()
-        t = time_plan(plan, stream)
-        out[what] = t / reps
-    return out
-
-
-KERNEL_NAMES = {"fused": "bgmv_fused_kernel", "group": "group_kernel",
-                "shrink": "shrink_items_kernel", "expand": "expand_items_kernel"}
-SEG_KERNEL_NAMES = {"shrink": "sgmv_shrink", "expand": "sgmv_expand"}
-
-
-def kernel_bytes(p, what):
-    by = algorithmic_bytes(p)
-    if what == "fused":
-        return by["shrink"] + by["expand"]
-    return by[what]
-
-
-def roofline_entry(p, ktimes, peak, peak_kind):
+def roofline_entry(p, ktimes, peak, peak_kind, fused_fits):
+    """Roofline of the dominant (longest) call of the step."""
     dom = max((k for k in ktimes if k != "group"), key=lambda k: ktimes[k])
-    ach = kernel_bytes(p, dom) / ktimes[dom] / 1e9
-    name = (SEG_KERNEL_NAMES if p.segmented else KERNEL_NAMES)[dom]
-    return {"bound": "hbm", "kernel": name, "achieved": round(ach, 1), "peak": peak,
+    ach = call_bytes(p, dom) / ktimes[dom] / 1e9
+    names = kernels_of(p, dom, fused_fits)
+    return {"bound": "hbm", "kernel": "+".join(names), "achieved": round(ach, 1), "peak": peak,
             "peak_kind": peak_kind, "unit": "GB/s", "frac": round(ach / peak, 4),
-            "traffic": profile_traffic(name),
-            "algorithmic_bytes": kernel_bytes(p, dom),
+            "traffic": profile_traffic(names[-1], p.name) if len(names) == 1 else None,
+            "algorithmic_bytes": call_bytes(p, dom),
             "us_per_launch": round(ktimes[dom] * 1e6, 3)}
 
 
@@ -529,125 +587,68 @@ def config_label(p):
             f"{W.DTYPE_NAME[p.dtype]} scale={p.scale}")
 
 
-def run_ours(args):
-    ws, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    init_dist(ws, "nccl")
-    dev = torch.device("cuda", local)
-    from gather_matmul_b200 import ops
-    ops.build_info()   # loads the library or fails loudly
-
-    probs = W.config(args.config)
-    p = probs[0]
-    if rank:   # data parallel: every rank serves its own batch of the same shape
-        p = W.make_problem(p.name, p.dtype, p.T, p.D, p.r, p.S, p.d_out, p.scale,
-                           seed=1000 * rank + args.config,
-                           idx_kind={2: "uniform", 1: "uniform_neg", 5: "zipf"}.get(args.config, "frac_neg"),
-                           frac_neg=0.25 if args.config == 3 else 0.10,
-                           segments=(p.seg_starts, p.seg_adapter) if p.segmented else None)
-    stream = torch.cuda.Stream(device=dev)
-    sets, runner, plan = measure_config(p, args.steps, args.warmup, stream)
-    peak, peak_kind = measured_peaks()
-
-    sampler = ClockSampler(local).start() if rank == 0 else None
-    time.sleep(0.2)
-    barrier(ws)
-    torch.cuda.synchronize()
-    elapsed = time_plan(plan, stream)
-    barrier(ws)
-    torch.cuda.synchronize()
-    kt = kernel_times(p, sets, stream, reps=min(args.steps, 2048))
-    clocks = sampler.stop() if sampler is not None else None
-
-    el_max = max_over_ranks(elapsed, ws, dev)
-    tokens_all = sum_over_ranks(p.T * args.steps, ws, dev)
-    value = tokens_all / el_max
+def workload_numbers(p, t_step, kt, peak, tf_peak, fused_fits, launches):
+    """Step and per-call figures of one projection: times, throughput, and the
+    fractions of the HBM roofline (algorithmic bytes / time / measured copy
+    bandwidth), of the tensor roofline (contraction FLOPs / time / bf16
+    peak), and of the slower of the two."""
     by = algorithmic_bytes(p)
-
-    e2e_steps = max(3, min(args.steps, 2000))
-    e2e_t, h2d, d2h = e2e_measure(p, sets, e2e_steps, 3, stream)
-    e2e_t = max_over_ranks(e2e_t, ws, dev)
-    e2e_val = sum_over_ranks(p.T * e2e_steps, ws, dev) / e2e_t
-
-    if rank != 0:
-        barrier(ws)
-        return
-    line = {
-        "metric": "LoRA shrink+expand tokens/s (achieved HBM GB/s and % of B200 roofline alongside)",
-        "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(el_max / args.steps * 1e3, 6),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": W.DTYPE_NAME[p.dtype], "data": "synthetic (seeded normal inputs, random adapters)",
-        "config": {"workload": config_label(p),
-                   "step": ("segment shrink + expand" if p.segmented else
-                            "group-by-slot + shrink + expand in one fused launch" if fused(p)
-                            else "group-by-slot + shrink + expand (3 launches)"),
-                   "l2": f"inputs larger than L2: {len(sets)} rotating input sets, "
-                         f"{sum(s.nbytes() for s in sets) / 1e6:.0f} MB > {L2_BYTES / 1e6:.0f} MB",
-                   "graph": "K steps replayed from CUDA graphs of up to 64 steps",
-                   "parallelism": f"dp{ws} independent replicas"},
-        "achieved_gbs_step": round(by["step"] * args.steps * ws / el_max / 1e9, 1),
-        "roofline": roofline_entry(p, kt, peak, peak_kind),
-        "kernel_us": {k: round(v * 1e6, 3) for k, v in kt.items()},
-        "gpu_launches": launches_per(p) * args.steps,
-        "e2e": {"value": round(e2e_val, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "clocks": clocks,
+    fl = algorithmic_flops(p)
+    Ta, U = active_stats(p)
+    return {
+        "workload": config_label(p),
+        "us_per_step": round(t_step * 1e6, 3),
+        "tokens_per_s": round(p.T / t_step, 1),
+        "active_tokens": Ta, "slots_used": U,
+        "launches_per_step": launches,
+        "gbs_step": round(by["step"] / t_step / 1e9, 1),
+        "frac_step": round(by["step"] / t_step / 1e9 / peak, 4),
+        "calls": {k: {"kernels": kernels_of(p, k, fused_fits),
+                      "us": round(v * 1e6, 3),
+                      "bytes": call_bytes(p, k),
+                      "gbs": round(call_bytes(p, k) / v / 1e9, 1),
+                      "frac_hbm": round(call_bytes(p, k) / v / 1e9 / peak, 4),
+                      "tensor_frac": round(call_flops(p, k) / v / 1e12 / tf_peak, 4)}
+                  for k, v in kt.items()},
+        "tflops_step": round(fl / t_step / 1e12, 2),
+        "tensor_frac_step": round(fl / t_step / 1e12 / tf_peak, 4),
+        "roofline_frac_step": round(max(fl / (tf_peak * 1e12), by["step"] / (peak * 1e9))
+                                    / t_step, 4),
+        "frac_step_vs_8tbs": round(by["step"] / t_step / 8e12, 4),
+        "bytes": by,
     }
-    if ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(p, budget_s=args.cpu_seconds)
-    if args.detail:
-        line["detail"] = detail_all(args, stream, peak, peak_kind)
-    print(json.dumps(line), flush=True)
-    barrier(ws)
 
 
-def detail_all(args, stream, peak, peak_kind):
-    """Per-projection numbers of every workload (not the headline line)."""
+def measure_workload(p, stream, reps, peak, tf_peak):
+    sets = make_sets(p)
+    ff = fused(p)
+    launches = launches_per_step(p, sets[0], stream)
+    kt = kernel_times(p, sets, stream, reps, ff)
+    t = warm_then_time(GraphRunner(p, sets, stream, "step"), reps) / reps
+    out = workload_numbers(p, t, kt, peak, tf_peak, ff, launches)
+    out["l2"] = f"{len(sets)} rotating input sets, {sum(s.nbytes() for s in sets) / 1e6:.0f} MB"
+    del sets
+    torch.cuda.empty_cache()
+    return out
+
+
+def configs_block(stream, peak, tf_peak, reps=256):
+    """Every workload: each projection's numbers, plus the three fused-slice
+    projections of one decoder layer summed."""
     out = {}
     layer = []
-    tf_peak = measured_bf16_tflops()
     for n in (1, 2, 3, 4, 5):
         for p in W.config(n):
-            sets = make_sets(p, extra_copies=True)
-            reps = 256
-            kt = kernel_times(p, sets, stream, reps)
-            r = GraphRunner(p, sets, stream, "step")
-            plan = r.prepare(reps)
-            with torch.cuda.stream(stream):
-                GraphRunner.run(r.prepare(min(reps, 64)))
-            t = time_plan(plan, stream) / reps
-            by = algorithmic_bytes(p)
-            fl = algorithmic_flops(p)
-            out[f"cfg{n}:{p.name}"] = {
-                "us_per_step": round(t * 1e6, 3),
-                "tokens_per_s": round(p.T / t, 1),
-                "gbs_step": round(by["step"] / t / 1e9, 1),
-                "frac_step": round(by["step"] / t / 1e9 / peak, 4),
-                "kernel_us": {k: round(v * 1e6, 3) for k, v in kt.items()},
-                "kernel_gbs": {k: round(kernel_bytes(p, k) / v / 1e9, 1) for k, v in kt.items()},
-                "kernel_frac": {k: round(kernel_bytes(p, k) / v / 1e9 / peak, 4)
-                                for k, v in kt.items()},
-                "tflops_step": round(fl / t / 1e12, 2),
-                # fraction of the tensor roofline, and of the slower of the two
-                # rooflines (contraction FLOPs at the bf16 peak, bytes at HBM)
-                "tensor_frac_step": round(fl / t / 1e12 / tf_peak, 4),
-                "roofline_frac_step": round(max(fl / (tf_peak * 1e12), by["step"] / (peak * 1e9))
-                                            / t, 4),
-                "frac_step_vs_8tbs": round(by["step"] / t / 8e12, 4),
-                "bytes": by,
-            }
+            r = measure_workload(p, stream, reps, peak, tf_peak)
+            out[f"cfg{n}:{p.name}"] = r
             if n == 3:
-                layer.append((t, by["step"], p.T))
-            del sets
-            torch.cuda.empty_cache()
-    # the three fused-slice projections of one decoder layer, back to back
+                layer.append((r["us_per_step"] * 1e-6, r["bytes"]["step"], p.T))
     t3 = sum(v[0] for v in layer)
     b3 = sum(v[1] for v in layer)
     out["cfg3:layer_sum"] = {"us_per_layer": round(t3 * 1e6, 3),
                              "tokens_per_s": round(layer[0][2] / t3, 1),
-                             "gbs": round(b3 / t3 / 1e9, 1), "frac": round(b3 / t3 / 1e9 / peak, 4)}
-    out["idle_call_us"] = idle_call_us()
+                             "gbs": round(b3 / t3 / 1e9, 1),
+                             "frac_hbm": round(b3 / t3 / 1e9 / peak, 4)}
     return out
 
 
@@ -683,6 +684,99 @@ def idle_call_us(calls=2000):
         fn(*args)
     out["c_abi"] = round((time.perf_counter() - t0) / calls * 1e6, 3)
     return out
+
+
+def run_ours(args):
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    init_dist(ws, "nccl")
+    dev = torch.device("cuda", local)
+    from gather_matmul_b200 import ops
+    ops.build_info()   # loads the library or fails loudly
+
+    p = W.config(args.config)[0]
+    if rank:   # data parallel: every rank serves its own batch of the same shape
+        p = W.make_problem(p.name, p.dtype, p.T, p.D, p.r, p.S, p.d_out, p.scale,
+                           seed=1000 * rank + args.config,
+                           idx_kind={2: "uniform", 1: "uniform_neg", 5: "zipf"}.get(args.config, "frac_neg"),
+                           frac_neg=0.25 if args.config == 3 else 0.10,
+                           segments=(p.seg_starts, p.seg_adapter) if p.segmented else None)
+    stream = torch.cuda.Stream(device=dev)
+    peak, peak_kind = measured_peaks()
+    tf_peak = measured_bf16_tflops()
+    sets = make_sets(p)
+    l2_desc = (f"inputs larger than L2: step k runs on input set k mod {len(sets)}, "
+               f"{sum(d.nbytes() for d in sets) / 1e6:.0f} MB in all > {L2_BYTES / 1e6:.0f} MB")
+    ff = fused(p)
+    launches = launches_per_step(p, sets[0], stream)
+    runner = GraphRunner(p, sets, stream, "step")
+    plan = runner.prepare(args.steps)
+    # warm-up: W untimed steps, and the exact timed graphs replayed once
+    runner.run(runner.prepare(args.warmup))
+    runner.run(plan)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local).start() if rank == 0 else None
+    time.sleep(0.2)
+    barrier(ws)
+    torch.cuda.synchronize()
+    elapsed = time_plan(runner, plan)
+    barrier(ws)
+    torch.cuda.synchronize()
+    reps = max(256, args.steps)
+    kt = kernel_times(p, sets, stream, reps, ff)
+
+    el_max = max_over_ranks(elapsed, ws, dev)
+    tokens_all = sum_over_ranks(p.T * args.steps, ws, dev)
+    value = tokens_all / el_max
+    by = algorithmic_bytes(p)
+
+    e2e_t, e2e_n, h2d, d2h = e2e_measure(p, sets, args.steps, 3, stream)
+    e2e_t = max_over_ranks(e2e_t, ws, dev)
+    e2e_val = sum_over_ranks(p.T * e2e_n, ws, dev) / e2e_t
+    del sets, runner, plan
+    torch.cuda.empty_cache()
+    blocks = None
+    if ws == 1 and not args.no_configs:
+        blocks = configs_block(stream, peak, tf_peak)
+    clocks = sampler.stop() if sampler is not None else None
+
+    if rank != 0:
+        barrier(ws)
+        return
+    line = {
+        "metric": "LoRA shrink+expand tokens/s (achieved HBM GB/s and % of B200 roofline alongside)",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(el_max / args.steps * 1e3, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": W.DTYPE_NAME[p.dtype], "data": "synthetic (seeded normal inputs, random adapters)",
+        "config": {"workload": config_label(p),
+                   "step": ("segment shrink + expand" if p.segmented else
+                            "one lora_bgmv call: group-by-slot + shrink + expand, "
+                            + ("one fused launch" if ff else f"{launches} launches")),
+                   "l2": l2_desc,
+                   "graph": "K steps replayed from CUDA graphs of up to 64 steps, "
+                            "the same graphs replayed once untimed first",
+                   "parallelism": f"dp{ws} independent replicas"},
+        "active_tokens_per_s": round(active_stats(p)[0] * args.steps * ws / el_max, 1),
+        "achieved_gbs_step": round(by["step"] * args.steps * ws / el_max / 1e9, 1),
+        "frac_step": round(by["step"] * args.steps * ws / el_max / 1e9 / peak, 4),
+        "roofline": roofline_entry(p, kt, peak, peak_kind, ff),
+        "kernel_us": {k: round(v * 1e6, 3) for k, v in kt.items()},
+        "kernel_reps": reps,
+        "gpu_launches": launches * args.steps,
+        "e2e": {"value": round(e2e_val, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_n,
+                "seconds": round(e2e_t, 4)},
+        "clocks": clocks,
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(p, budget_s=args.cpu_seconds)
+    if blocks is not None:
+        blocks["idle_call_us"] = idle_call_us()
+        line["configs"] = blocks
+    print(json.dumps(line), flush=True)
+    barrier(ws)
 
 
 # --------------------------------------------------------------------------
@@ -738,11 +832,13 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--config", type=int, default=5, choices=[1, 2, 3, 4, 5],
+                    help="headline workload (default 5: the large mixed batch)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--detail", action="store_true", help="add every workload's numbers")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="leave out the per-workload block")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=60.0)

@@ -29,10 +29,10 @@ SIGNATURES = {
     "lora_workspace_bytes": (_sz, [_i32, _i32]),
     "lora_workspace_reset": (_i32, [_vp, _sz, _vp]),
     "lora_group": (_i32, [_i32, _i32, _vp, _vp, _sz, _vp]),
-    "lora_shrink": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _i32, _vp,
-                           _sz, _vp]),
-    "lora_expand": (_i32, [_i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _vp, _i64,
-                           _vp, _i32, _vp, _sz, _vp]),
+    "lora_shrink": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _i32,
+                           _vp, _sz, _vp]),
+    "lora_expand": (_i32, [_i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _f32, _vp,
+                           _i64, _vp, _i32, _vp, _sz, _vp]),
     "lora_shrink_segment": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp,
                                    _i32, _vp, _i32, _vp, _sz, _vp]),
     "lora_expand_segment": (_i32, [_i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _vp,
@@ -45,6 +45,7 @@ SIGNATURES = {
                                    _vp, _i32, _vp]),
     "lora_status_string": (ctypes.c_char_p, [_i32]),
     "lora_build_info": (ctypes.c_char_p, []),
+    "lora_launch_count": (ctypes.c_ulonglong, []),
 }
 
 _lib = None

@@ -101,7 +101,16 @@ shrink_items_kernel(const ShrinkArgs a) {
     const int4 it = items[item];
     const int slot = it.x, nt = it.z - it.y;
     __syncthreads();   // previous item's readers of stok / cpart are done
-    if (tid < nt) stok[tid] = (it.w & kItemDirect) ? it.y + tid : perm[it.y + tid];
+    if (tid < nt) {
+      // a token of a per-token grouping whose index disagrees with its group
+      // (stale workspace) is skipped (-1) and counted once per item
+      int tok = (it.w & kItemDirect) ? it.y + tid : perm[it.y + tid];
+      if (!(it.w & kItemDirect) && !grouped_row_ok(a.idx, tok, slot, a.S)) {
+        if (crank == 0 && blockIdx.y == 0) count_bad_meta(a.meta, 1);
+        tok = -1;
+      }
+      stok[tid] = tok;
+    }
     for (int e = tid; e < kWarps * kItemTokens * kJR; e += kThreads)
       (&sacc[0][0][0])[e] = 0.f;
     __syncthreads();
@@ -109,7 +118,7 @@ shrink_items_kernel(const ShrinkArgs a) {
     if (slot < 0) {          // tokens without an adapter: buf rows are zero
       if (crank == 0)
         for (int e = tid; e < nt * kJR; e += kThreads)
-          bufs[(size_t)stok[e / kJR] * r + j0 + e % kJR] = 0.f;
+          if (stok[e / kJR] >= 0) bufs[(size_t)stok[e / kJR] * r + j0 + e % kJR] = 0.f;
       continue;
     }
 
@@ -128,8 +137,8 @@ shrink_items_kernel(const ShrinkArgs a) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int k = k0 + q;
-          xu[q] = (inb && k < nt) ? ldg_nc(x + (size_t)stok[k] * a.ldx + col)
-                                  : make_uint4(0, 0, 0, 0);
+          xu[q] = (inb && k < nt && stok[k] >= 0) ? ldg_nc(x + (size_t)stok[k] * a.ldx + col)
+                                                  : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -162,7 +171,7 @@ shrink_items_kernel(const ShrinkArgs a) {
     if (CL == 1) {
       __syncthreads();
       for (int e = tid; e < nt * kJR; e += kThreads)
-        bufs[(size_t)stok[e / kJR] * r + j0 + e % kJR] = cpart[e];
+        if (stok[e / kJR] >= 0) bufs[(size_t)stok[e / kJR] * r + j0 + e % kJR] = cpart[e];
     } else {
       cluster.sync();      // every CTA's cpart is complete
       const int per = (nt * kJR + CL - 1) / CL;
@@ -170,7 +179,7 @@ shrink_items_kernel(const ShrinkArgs a) {
       for (int e = e0 + tid; e < e1; e += kThreads) {
         float s = 0.f;
         for (int q = 0; q < CL; ++q) s += cluster.map_shared_rank(cpart, q)[e];
-        bufs[(size_t)stok[e / kJR] * r + j0 + e % kJR] = s;
+        if (stok[e / kJR] >= 0) bufs[(size_t)stok[e / kJR] * r + j0 + e % kJR] = s;
       }
       cluster.sync();      // no CTA reuses cpart while a peer still reads it
     }
@@ -221,10 +230,19 @@ expand_items_kernel(const ExpandArgs a) {
     const float* bsl = a.buf + (size_t)slice * a.buf_slice_stride;
 
     __syncthreads();   // previous unit's readers of sbuf / stok are done
-    if (tid < nt) stok[tid] = (it.w & kItemDirect) ? it.y + tid : perm[it.y + tid];
+    if (tid < nt) {
+      // tokens whose index disagrees with their group (stale workspace) are
+      // neither read nor written; counted once per item
+      int tok = (it.w & kItemDirect) ? it.y + tid : perm[it.y + tid];
+      if (!(it.w & kItemDirect) && !grouped_row_ok(a.idx, tok, slot, a.S)) {
+        if (ch == 0) count_bad_meta(a.meta, 1);
+        tok = -1;
+      }
+      stok[tid] = tok;
+    }
     __syncthreads();
     for (int e = tid; e < nt * R; e += kThreads)
-      sbuf[e / R][e % R] = bsl[(size_t)stok[e / R] * R + e % R];
+      sbuf[e / R][e % R] = stok[e / R] >= 0 ? bsl[(size_t)stok[e / R] * R + e % R] : 0.f;
     __syncthreads();
     if (!active) continue;
 
@@ -244,11 +262,12 @@ expand_items_kernel(const ExpandArgs a) {
       typename YV::T yv[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q)
-        if (k0 + q < nt) yv[q] = YV::load(ybase + (size_t)stok[k0 + q] * a.ldy);
+        if (k0 + q < nt && stok[k0 + q] >= 0) yv[q] = YV::load(ybase + (size_t)stok[k0 + q] * a.ldy);
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const int k = k0 + q;
         if (k >= nt) break;
+        if (stok[k] < 0) continue;
         float acc[CPL];
 #pragma unroll
         for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
@@ -296,7 +315,7 @@ cudaError_t shrink_dispatch(const ShrinkArgs& a, int max_items, cudaStream_t st)
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, shrink_items_kernel<E>, a);
+  return counted_launch(cudaLaunchKernelEx(&cfg, shrink_items_kernel<E>, a));
 }
 
 template <typename E, int R, int CPL>
@@ -305,7 +324,7 @@ cudaError_t expand_launch(const ExpandArgs& a, int max_items, cudaStream_t st) {
   int grid = units < kPersistentCtas ? (int)units : kPersistentCtas;
   if (grid < 1) grid = 1;
   expand_items_kernel<E, R, CPL><<<grid, kThreads, 0, st>>>(a);
-  return cudaGetLastError();
+  return counted_launch(cudaGetLastError());
 }
 
 template <typename E>

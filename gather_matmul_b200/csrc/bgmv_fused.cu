@@ -575,7 +575,7 @@ cudaError_t fused_launch(const FusedArgs& a, lora_dtype dt, cudaStream_t st) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, P);
+  return counted_launch(cudaLaunchKernelEx(&cfg, kern, P));
 }
 
 }  // namespace

@@ -132,4 +132,19 @@ __device__ __forceinline__ int checked_items(const char* meta, int T, int S) {
   return 0;
 }
 
+// Whether token `tok` really belongs to the group of a per-token grouping it
+// was placed in: idx[tok] == slot for an adapter's group, idx[tok] outside
+// [0, S) for the group of tokens without an adapter.  A grouping built from
+// another batch's indices (a stale workspace) fails this for every token
+// whose index changed, so the kernels skip those rows and count them instead
+// of computing them with the wrong adapter.
+__device__ __forceinline__ bool grouped_row_ok(const int32_t* idx, int tok, int slot, int S) {
+  const int v = idx[tok];
+  return slot >= 0 ? v == slot : (v < 0 || v >= S);
+}
+
+__device__ __forceinline__ void count_bad_meta(const char* meta, int n) {
+  atomicAdd(const_cast<int*>(&reinterpret_cast<const MetaHeader*>(meta)->bad_meta), n);
+}
+
 }  // namespace lora

@@ -231,14 +231,14 @@ cudaError_t launch_group(int T, int S, const int32_t* idx, void* meta, cudaStrea
                                        (int)smem);
   if (e != cudaSuccess) return e;
   group_kernel<<<1, kGroupThreads, smem, st>>>(T, S, idx, static_cast<char*>(meta));
-  return cudaGetLastError();
+  return counted_launch(cudaGetLastError());
 }
 
 cudaError_t launch_segment_items(int T, int S, int n_seg, const int32_t* seg_starts,
                                  const int32_t* seg_adapter, void* meta, cudaStream_t st) {
   segment_items_kernel<<<1, kGroupThreads, 0, st>>>(T, S, n_seg, seg_starts, seg_adapter,
                                                     static_cast<char*>(meta));
-  return cudaGetLastError();
+  return counted_launch(cudaGetLastError());
 }
 
 }  // namespace lora

@@ -14,6 +14,7 @@ struct ShrinkArgs {
   const void* x;
   int64_t ldx;
   const void* A[LORA_MAX_SLICES];
+  const int32_t* idx;       // per-token indices the grouping is checked against (null: segments)
   float* buf;
   int T, D, r, S, n_slices;
   const char* meta;
@@ -22,6 +23,7 @@ struct ShrinkArgs {
 struct ExpandArgs {
   const float* buf;
   int64_t buf_slice_stride;
+  const int32_t* idx;       // per-token indices the grouping is checked against (null: segments)
   const void* B[LORA_MAX_SLICES];
   int D_out[LORA_MAX_SLICES];
   int64_t y_col_off[LORA_MAX_SLICES];
@@ -58,6 +60,11 @@ struct FusedArgs {
   float scale;
   int pdl_early;            // A, B and idx may be read before the previous kernel ends
 };
+
+// Every kernel launch of the library passes its status through here, so that
+// lora_launch_count() reports how many launches (or stream-capture records)
+// the library has made.
+cudaError_t counted_launch(cudaError_t e);
 
 cudaError_t encode_tmap_2d(CUtensorMap* map, lora_dtype dt, const void* base, uint64_t inner,
                            uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,

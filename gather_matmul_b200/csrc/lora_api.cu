@@ -87,7 +87,16 @@ lora_status check_segments(int T, int n_seg, const int32_t* seg_starts,
 int max_items_tokens(int T, int S) { return T / kItemTokens + S + 2; }
 int max_items_segments(int T, int n_seg) { return T / kItemTokens + n_seg + 2; }
 
+std::atomic<unsigned long long> g_launches{0};
+
 }  // namespace
+
+namespace lora {
+cudaError_t counted_launch(cudaError_t e) {
+  if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
+}  // namespace lora
 
 extern "C" {
 
@@ -113,16 +122,18 @@ lora_status lora_group(int T, int S, const int32_t* idx, void* meta, size_t meta
 }
 
 lora_status lora_shrink(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
-                        const void* x, int64_t ldx, const void* const* A, float* buf,
-                        int has_active, const void* meta, size_t meta_bytes,
+                        const void* x, int64_t ldx, const void* const* A, const int32_t* idx,
+                        float* buf, int has_active, const void* meta, size_t meta_bytes,
                         lora_stream_t stream) {
   lora_status s = check_shrink(dtype, T, D, r, S, n_slices, x, ldx, A, buf, meta, meta_bytes);
   if (s != LORA_OK) return s;
   if (!has_active || T == 0) return LORA_OK;
+  if (idx == nullptr) return LORA_ERR_INVALID_ARG;
   ShrinkArgs a = {};
   a.x = x;
   a.ldx = ldx;
   for (int i = 0; i < n_slices; ++i) a.A[i] = A[i];
+  a.idx = idx;
   a.buf = buf;
   a.T = T; a.D = D; a.r = r; a.S = S; a.n_slices = n_slices;
   a.meta = static_cast<const char*>(meta);
@@ -137,10 +148,11 @@ lora_status lora_shrink(lora_dtype dtype, int T, int D, int r, int S, int n_slic
 
 static void fill_expand(ExpandArgs& a, int T, int r, int S, int n_slices, const float* buf,
                         int64_t buf_slice_stride, const void* const* B, const int32_t* D_out,
-                        float scale, void* y, int64_t ldy, const int64_t* y_col_off,
-                        const void* meta) {
+                        const int32_t* idx, float scale, void* y, int64_t ldy,
+                        const int64_t* y_col_off, const void* meta) {
   a.buf = buf;
   a.buf_slice_stride = buf_slice_stride;
+  a.idx = idx;
   for (int i = 0; i < n_slices; ++i) {
     a.B[i] = B[i];
     a.D_out[i] = D_out[i];
@@ -155,16 +167,17 @@ static void fill_expand(ExpandArgs& a, int T, int r, int S, int n_slices, const 
 
 lora_status lora_expand(lora_dtype dtype, int T, int r, int S, int n_slices,
                         const float* buf, int64_t buf_slice_stride, const void* const* B,
-                        const int32_t* D_out, float scale, void* y, int64_t ldy,
-                        const int64_t* y_col_off, int has_active, const void* meta,
+                        const int32_t* D_out, const int32_t* idx, float scale, void* y,
+                        int64_t ldy, const int64_t* y_col_off, int has_active, const void* meta,
                         size_t meta_bytes, lora_stream_t stream) {
   lora_status s = check_expand(dtype, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, y,
                                ldy, y_col_off, meta, meta_bytes);
   if (s != LORA_OK) return s;
   if (!has_active || T == 0) return LORA_OK;
+  if (idx == nullptr) return LORA_ERR_INVALID_ARG;
   ExpandArgs a = {};
-  fill_expand(a, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, scale, y, ldy, y_col_off,
-              meta);
+  fill_expand(a, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, idx, scale, y, ldy,
+              y_col_off, meta);
   cudaGetLastError();
   if (grouped_tc_preferred(T, r, S)) {
     cudaError_t e = launch_expand_grouped_tc(dtype, a, (cudaStream_t)stream);
@@ -217,8 +230,8 @@ lora_status lora_expand_segment(lora_dtype dtype, int T, int r, int S, int n_sli
   if (s != LORA_OK) return s;
   if (!has_active || T == 0) return LORA_OK;
   ExpandArgs a = {};
-  fill_expand(a, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, scale, y, ldy, y_col_off,
-              meta);
+  fill_expand(a, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, nullptr, scale, y, ldy,
+              y_col_off, meta);
   SegArgs sg = {seg_starts, seg_adapter, n_seg};
   cudaStream_t st = (cudaStream_t)stream;
   cudaGetLastError();
@@ -282,10 +295,10 @@ lora_status lora_bgmv(lora_dtype dtype, int T, int D, int r, int S, int n_slices
   cudaGetLastError();
   s = lora_group(T, S, idx, meta, meta_bytes, stream);
   if (s != LORA_OK) return s;
-  s = lora_shrink(dtype, T, D, r, S, n_a, x, ldx, A, buf, 1, meta, meta_bytes, stream);
+  s = lora_shrink(dtype, T, D, r, S, n_a, x, ldx, A, idx, buf, 1, meta, meta_bytes, stream);
   if (s != LORA_OK) return s;
   return lora_expand(dtype, T, r, S, n_slices, buf, shared_A ? 0 : (int64_t)T * r, B, D_out,
-                     scale, y, ldy, y_col_off, 1, meta, meta_bytes, stream);
+                     idx, scale, y, ldy, y_col_off, 1, meta, meta_bytes, stream);
 }
 
 int lora_bgmv_launches(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
@@ -324,7 +337,11 @@ const char* lora_status_string(lora_status status) {
   return "LORA_ERR_UNKNOWN";
 }
 
-const char* lora_build_info(void) { return "liblora_b200 sm_100a 0.1"; }
+const char* lora_build_info(void) { return "liblora_b200 sm_100a 0.2"; }
+
+unsigned long long lora_launch_count(void) {
+  return g_launches.load(std::memory_order_relaxed);
+}
 
 }  // extern "C"
 
@@ -397,6 +414,7 @@ extern "C" LORA_API lora_status lora_shrink_noalloc(lora_dtype dtype, int T, int
   a.x = x;
   a.ldx = ldx;
   for (int i = 0; i < n_slices; ++i) a.A[i] = A[i];
+  a.idx = idx;
   a.buf = buf;
   a.T = T; a.D = D; a.r = r; a.S = S; a.n_slices = n_slices;
   a.meta = static_cast<const char*>(scratch);

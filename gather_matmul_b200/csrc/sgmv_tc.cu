@@ -141,6 +141,7 @@ struct ShrinkTCParams {
   int n_seg;
   float* buf;
   const int32_t* perm;                   // row p of a tile is token perm[p]; null = identity
+  const int32_t* idx;                    // per-token indices checked against the grouping
   int implicit_slots;                    // > 0: segment g is slot g (per-token grouping)
   int T, D, S, n_slices, KS;
   int* bad_index;
@@ -210,10 +211,22 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   const int m0 = sinfo[1], valid = sinfo[2], adapter = sinfo[3];
   float* bufs = P.buf + (size_t)slice * P.T * R;
   const int32_t* perm = P.perm;
-  auto token = [&](int p) { return perm ? perm[p] : p; };
+  // token of tile row p, or -1 when a per-token grouping placed a token whose
+  // index disagrees with the group (stale workspace): that row is not written,
+  // and the writer of the row counts it
+  auto token = [&](int p, bool count) {
+    if (!perm) return p;
+    const int t = perm[p];
+    if (grouped_row_ok(P.idx, t, adapter, P.S)) return t;
+    if (count && slice == 0) atomicAdd(P.bad_meta, 1);
+    return -1;
+  };
   if (adapter < 0 || adapter >= P.S) {        // no adapter: zero rows (rank 0 writes them)
     if (kr == 0)
-      for (int e = tid; e < valid * R; e += kShrThreads) bufs[(size_t)token(m0 + e / R) * R + e % R] = 0.f;
+      for (int e = tid; e < valid * R; e += kShrThreads) {
+        const int t = token(m0 + e / R, e % R == 0);
+        if (t >= 0) bufs[(size_t)t * R + e % R] = 0.f;
+      }
     return;
   }
 
@@ -312,8 +325,9 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
     }
   }
   if (KS == 1) {
-    if (has_row && m < valid) {
-      float4* row = reinterpret_cast<float4*>(bufs + (size_t)token(m0 + m) * R);
+    const int t = has_row && m < valid ? token(m0 + m, true) : -1;
+    if (t >= 0) {
+      float4* row = reinterpret_cast<float4*>(bufs + (size_t)t * R);
 #pragma unroll
       for (int q = 0; q < R / 4; ++q) row[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
@@ -337,7 +351,8 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
       float sum = 0.f;
       for (int q = 0; q < KS; ++q) sum += recv[(size_t)(q * rows + lm) * L::kPitch + j];
       const int mm = kr * rows + lm;
-      if (mm < valid) bufs[(size_t)token(m0 + mm) * R + j] = sum;
+      const int t = mm < valid ? token(m0 + mm, j == 0) : -1;
+      if (t >= 0) bufs[(size_t)t * R + j] = sum;
     }
   }
   ptx::tc_fence_before();
@@ -385,6 +400,7 @@ struct ExpandTCParams {
   const int32_t* seg_adapter;
   int n_seg;
   const int32_t* perm;                   // row p of a tile is token perm[p]; null = identity
+  const int32_t* idx;                    // per-token indices checked against the grouping
   int implicit_slots;                    // > 0: segment g is slot g (per-token grouping)
   int T, S, n_slices;
   float scale;
@@ -681,7 +697,14 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
         // are free without waiting, then the hi / lo rows, so that the buf
         // reads overlap those loads
         const int m = lt;
-        const int tok = m < rn.valid ? (P.perm ? P.perm[rn.m0 + m] : rn.m0 + m) : -1;
+        // sTok: the row's token; -1 past the tile; -2 - token for a token whose
+        // index disagrees with its group (stale workspace): still a valid row
+        // address for the gathers, but never written back (counted here)
+        int tok = m < rn.valid ? (P.perm ? P.perm[rn.m0 + m] : rn.m0 + m) : -1;
+        if (tok >= 0 && P.perm && !grouped_row_ok(P.idx, tok, rn.adapter, P.S)) {
+          if (rn.j0 == 0) atomicAdd(P.bad_meta, 1);
+          tok = -2 - tok;
+        }
         sTok[hb * kTM + m] = tok;
         asm volatile("bar.sync 4, 128;" ::: "memory");   // every row's token is known
         const int* toks = sTok + hb * kTM;
@@ -718,7 +741,10 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
               const int g = o >> 1, h = o & 1;
               int rr[4];
 #pragma unroll
-              for (int q = 0; q < 4; ++q) rr[q] = toks[4 * g + q < rn.valid ? 4 * g + q : 4 * g];
+              for (int q = 0; q < 4; ++q) {
+                const int t = toks[4 * g + q < rn.valid ? 4 * g + q : 4 * g];
+                rr[q] = t >= 0 ? t : -2 - t;
+              }
               ptx::tma_gather4(ys + h * L::kYHalf + g * 512, &P.tmYg, (int)(ycol0 + n0 + 64 * h),
                                rr[0], rr[1], rr[2], rr[3], &full[s]);
             }
@@ -904,7 +930,7 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
               for (int i = 0; i < 8; ++i) {
                 const int lr = 4 * i + (lane >> 3);
                 const int tk = __shfl_sync(0xffffffffu, tok, lr);
-                if (q * 32 + lr < rn.valid && col_ok)
+                if (q * 32 + lr < rn.valid && col_ok && tk >= 0)
                   *reinterpret_cast<uint4*>(ycol + (size_t)tk * P.ldy + n0 + 64 * h + 8 * ch) = v[i];
               }
               ptx::fence_proxy_async_smem();
@@ -956,7 +982,7 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
             for (int it = 0; it < 8; ++it) {
               const int e = gl + 128 * it;
               const int mr = e >> 4, hh = (e >> 3) & 1, ch = e & 7;
-              if (mr < rn.valid && 64 * hh + 8 * ch < nn)
+              if (mr < rn.valid && 64 * hh + 8 * ch < nn && toks[mr] >= 0)
                 *reinterpret_cast<uint4*>(ycol + (size_t)toks[mr] * P.ldy + n0 + 64 * hh + 8 * ch) =
                     v[it];
             }
@@ -1026,6 +1052,7 @@ cudaError_t shrink_tc_launch(const ShrinkArgs& a, const SegArgs& sg, lora_dtype 
   P.n_seg = sg.n_seg;
   P.buf = a.buf;
   P.perm = perm;
+  P.idx = a.idx;
   P.implicit_slots = implicit_slots;
   P.T = a.T;
   P.D = a.D;
@@ -1078,7 +1105,7 @@ cudaError_t shrink_tc_launch(const ShrinkArgs& a, const SegArgs& sg, lora_dtype 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, P);
+  return counted_launch(cudaLaunchKernelEx(&cfg, kern, P));
 }
 
 template <typename E, int R>
@@ -1113,6 +1140,7 @@ cudaError_t expand_tc_launch(const ExpandArgs& a, const SegArgs& sg, lora_dtype 
   P.seg_adapter = sg.seg_adapter;
   P.n_seg = sg.n_seg;
   P.perm = perm;
+  P.idx = a.idx;
   P.implicit_slots = implicit_slots;
   P.T = a.T;
   P.S = a.S;
@@ -1130,7 +1158,7 @@ cudaError_t expand_tc_launch(const ExpandArgs& a, const SegArgs& sg, lora_dtype 
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kExpThreads, smem, st>>>(P);
-  return cudaGetLastError();
+  return counted_launch(cudaGetLastError());
 }
 
 }  // namespace

@@ -7,10 +7,17 @@ computation runs in the library's CUDA kernels; torch supplies device memory
 and streams.
 
   group(idx, S, meta)                          per-batch group-by-slot metadata
-  shrink(x, A, buf, meta)                      buf[i] = per-token x . A_i[idx]^T
-  expand(buf, B, y, meta, scale)               y[:, slice_i] += scale buf_i . B_i[idx]^T
+  shrink(x, A, idx, buf, meta)                 buf[i] = per-token x . A_i[idx]^T
+  expand(buf, B, idx, y, meta, scale)          y[:, slice_i] += scale buf_i . B_i[idx]^T
+  bgmv(x, A, B, idx, y, buf, meta, scale)      group + shrink + expand in one call
   shrink_segment / expand_segment              the same with segments
   check_errors(meta)                           device-side bad-index report
+
+has_active: the per-token calls take the host flag of the C ABI.  Left as
+None, it is derived from `idx_host` (a host copy of the batch's indices, as a
+serving loop has before it moves them to the device) when one is given: no
+index in [0, S) means no LoRA work at all, so nothing is enqueued.  Without a
+host copy the call runs, and the kernels skip tokens without an adapter.
 """
 import ctypes
 from typing import Optional, Sequence
@@ -52,6 +59,31 @@ def _dtype(t):
     return _DT[t.dtype]
 
 
+def active_from_host(idx_host, S: int) -> bool:
+    """Whether any index of a host copy of a batch's indices selects a slot
+    in [0, S)."""
+    if isinstance(idx_host, torch.Tensor):
+        if idx_host.is_cuda:
+            raise ValueError("idx_host must be a host tensor or array")
+        idx_host = idx_host.numpy()
+    import numpy as np
+    a = np.asarray(idx_host)
+    return bool(np.any((a >= 0) & (a < S)))
+
+
+def _active(has_active, idx_host, S):
+    if has_active is not None:
+        return int(bool(has_active))
+    if idx_host is not None:
+        return int(active_from_host(idx_host, S))
+    return 1
+
+
+def _check_idx(idx, T):
+    if idx.dtype != torch.int32 or not idx.is_contiguous() or idx.numel() != T:
+        raise TypeError("idx must be a contiguous int32 tensor of one index per token")
+
+
 def workspace_bytes(T: int, S: int) -> int:
     return _lib.load().lora_workspace_bytes(int(T), int(S))
 
@@ -66,8 +98,7 @@ def workspace(T: int, S: int, device="cuda") -> torch.Tensor:
 
 def group(idx: torch.Tensor, S: int, meta: torch.Tensor, stream=None):
     """Group-by-slot metadata of one batch's int32 adapter indices (-1 = none)."""
-    if idx.dtype != torch.int32 or not idx.is_contiguous():
-        raise TypeError("idx must be a contiguous int32 tensor")
+    _check_idx(idx, idx.numel())
     _check("lora_group", _lib.load().lora_group(idx.numel(), int(S), _ptr(idx), _ptr(meta),
                                                 meta.numel(), _stream(stream)))
 
@@ -78,16 +109,19 @@ def _xinfo(x):
     return x.shape[0], x.shape[1], (x.stride(0) if x.numel() > 0 else x.shape[1])
 
 
-def shrink(x: torch.Tensor, A: Sequence[torch.Tensor], buf: torch.Tensor, meta: torch.Tensor,
-           has_active: bool = True, stream=None) -> torch.Tensor:
+def shrink(x: torch.Tensor, A: Sequence[torch.Tensor], idx: torch.Tensor, buf: torch.Tensor,
+           meta: torch.Tensor, has_active: Optional[bool] = None, idx_host=None,
+           stream=None) -> torch.Tensor:
     """buf[i, t, :] = x[t] . A[i][idx[t]]^T (0 for tokens without an adapter).
 
-    A: list of [S, r, D] stacks; buf: float32 [len(A), T, r]; meta from group()."""
+    A: list of [S, r, D] stacks; idx: the device int32 indices that group()
+    grouped into meta; buf: float32 [len(A), T, r]."""
     T, D, ldx = _xinfo(x)
     S, r, _ = A[0].shape
+    _check_idx(idx, T)
     _check("lora_shrink", _lib.load().lora_shrink(
-        _dtype(x), T, D, r, S, len(A), _ptr(x), ldx, _ptrs(A), _ptr(buf), int(bool(has_active)),
-        _ptr(meta), meta.numel(), _stream(stream)))
+        _dtype(x), T, D, r, S, len(A), _ptr(x), ldx, _ptrs(A), _ptr(idx), _ptr(buf),
+        _active(has_active, idx_host, S), _ptr(meta), meta.numel(), _stream(stream)))
     return buf
 
 
@@ -110,23 +144,26 @@ def _expand_common(buf, B, y, y_col_off, buf_slice_stride):
     return T, ldy, S, r, n, d_out, off, int(buf_slice_stride)
 
 
-def expand(buf: torch.Tensor, B: Sequence[torch.Tensor], y: torch.Tensor, meta: torch.Tensor,
-           scale: float = 1.0, y_col_off=None, buf_slice_stride=None, has_active: bool = True,
-           stream=None) -> torch.Tensor:
+def expand(buf: torch.Tensor, B: Sequence[torch.Tensor], idx: torch.Tensor, y: torch.Tensor,
+           meta: torch.Tensor, scale: float = 1.0, y_col_off=None, buf_slice_stride=None,
+           has_active: Optional[bool] = None, idx_host=None, stream=None) -> torch.Tensor:
     """y[t, off_i:off_i+D_out_i] += scale * buf[i, t] . B[i][idx[t]]^T, in place.
 
-    B: list of [S, D_out_i, r]; buf: float32 [n, T, r] (or [T, r] shared by
-    every slice); y: [T, >= sum D_out] fp16/bf16."""
+    B: list of [S, D_out_i, r]; idx as for shrink(); buf: float32 [n, T, r]
+    (or [T, r] shared by every slice); y: [T, >= sum D_out] fp16/bf16."""
     T, ldy, S, r, n, d_out, off, stride = _expand_common(buf, B, y, y_col_off, buf_slice_stride)
+    _check_idx(idx, T)
     _check("lora_expand", _lib.load().lora_expand(
-        _dtype(y), T, r, S, n, _ptr(buf), stride, _ptrs(B), d_out, ctypes.c_float(scale),
-        _ptr(y), ldy, off, int(bool(has_active)), _ptr(meta), meta.numel(), _stream(stream)))
+        _dtype(y), T, r, S, n, _ptr(buf), stride, _ptrs(B), d_out, _ptr(idx),
+        ctypes.c_float(scale), _ptr(y), ldy, off, _active(has_active, idx_host, S), _ptr(meta),
+        meta.numel(), _stream(stream)))
     return y
 
 
 def bgmv(x: torch.Tensor, A: Sequence[torch.Tensor], B: Sequence[torch.Tensor], idx: torch.Tensor,
          y: torch.Tensor, buf: torch.Tensor, meta: torch.Tensor, scale: float = 1.0,
-         y_col_off=None, has_active: bool = True, pdl_early: bool = False, stream=None):
+         y_col_off=None, has_active: Optional[bool] = None, idx_host=None,
+         pdl_early: bool = False, stream=None):
     """group + shrink + expand of one batch in one call (one launch when the
     shape fits the fused kernel).  A: one stack per slice of B, or a single
     stack shared by every slice; buf: float32 [len(A), T, r] receives the
@@ -139,13 +176,12 @@ def bgmv(x: torch.Tensor, A: Sequence[torch.Tensor], B: Sequence[torch.Tensor], 
     if not shared and len(A) != n:
         raise ValueError("A must hold one stack per slice, or one shared stack")
     _, ldy, _, _, _, d_out, off, _ = _expand_common(buf, B, y, y_col_off, None)
-    if idx.dtype != torch.int32 or not idx.is_contiguous():
-        raise TypeError("idx must be a contiguous int32 tensor")
+    _check_idx(idx, T)
     flags = _lib.LORA_FLAG_PDL_EARLY if pdl_early else 0
     _check("lora_bgmv", _lib.load().lora_bgmv(
         _dtype(x), T, D, r, S, n, _ptr(x), ldx, _ptrs(A), int(shared), _ptrs(B), d_out,
-        ctypes.c_float(scale), _ptr(y), ldy, off, _ptr(buf), _ptr(idx), int(bool(has_active)),
-        flags, _ptr(meta), meta.numel(), _stream(stream)))
+        ctypes.c_float(scale), _ptr(y), ldy, off, _ptr(buf), _ptr(idx),
+        _active(has_active, idx_host, S), flags, _ptr(meta), meta.numel(), _stream(stream)))
     return y
 
 
@@ -185,8 +221,7 @@ def shrink_noalloc(x: torch.Tensor, A: Sequence[torch.Tensor], idx: torch.Tensor
     allocate; calls that overlap on the GPU race on that array."""
     T, D, ldx = _xinfo(x)
     S, r, _ = A[0].shape
-    if idx.dtype != torch.int32 or not idx.is_contiguous():
-        raise TypeError("idx must be a contiguous int32 tensor")
+    _check_idx(idx, T)
     _check("lora_shrink_noalloc", _lib.load().lora_shrink_noalloc(
         _dtype(x), T, D, r, S, len(A), _ptr(x), ldx, _ptrs(A), _ptr(idx), _ptr(buf),
         int(bool(has_active)), _stream(stream)))
@@ -201,3 +236,9 @@ def check_errors(meta: torch.Tensor, stream=None) -> int:
 
 def build_info() -> str:
     return _lib.load().lora_build_info().decode()
+
+
+def launch_count() -> int:
+    """Kernel launches the library has made in this process (a launch recorded
+    into a stream capture counts once)."""
+    return int(_lib.load().lora_launch_count())

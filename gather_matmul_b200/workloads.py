@@ -142,31 +142,34 @@ def prefill_segments(rng_seed, n_seq, seq_len, S):
 
 
 # The five workloads.  Each entry returns the list of projections that make
-# one step of that workload.
-def config(n: int) -> List[Problem]:
+# one step of that workload.  `dtype` draws the same workload in another
+# element type (same seeds and shapes).
+def config(n: int, dtype: Optional[int] = None) -> List[Problem]:
+    def dt(default):
+        return default if dtype is None else dtype
     if n == 1:   # tiny BGMV
-        return [make_problem("tiny_bgmv", F16, T=32, D=1024, r=8, S=4, d_out=[1024],
+        return [make_problem("tiny_bgmv", dt(F16), T=32, D=1024, r=8, S=4, d_out=[1024],
                              scale=1.0, seed=1, idx_kind="uniform_neg")]
     if n == 2:   # decode at a Llama-3-8B q_proj shape
-        return [make_problem("decode_q_proj", F16, T=256, D=4096, r=16, S=32,
+        return [make_problem("decode_q_proj", dt(F16), T=256, D=4096, r=16, S=32,
                              d_out=[4096], scale=2.0, seed=2, idx_kind="uniform")]
     if n == 3:   # fused-slice decode: qkv, gate_up, down
         return [
-            make_problem("decode_qkv", BF16, T=512, D=4096, r=64, S=8,
+            make_problem("decode_qkv", dt(BF16), T=512, D=4096, r=64, S=8,
                          d_out=[4096, 1024, 1024], seed=3, idx_kind="frac_neg",
                          frac_neg=0.25),
-            make_problem("decode_gate_up", BF16, T=512, D=4096, r=64, S=8,
+            make_problem("decode_gate_up", dt(BF16), T=512, D=4096, r=64, S=8,
                          d_out=[14336, 14336], seed=3, idx_kind="frac_neg",
                          frac_neg=0.25),
-            make_problem("decode_down", BF16, T=512, D=14336, r=64, S=8,
+            make_problem("decode_down", dt(BF16), T=512, D=14336, r=64, S=8,
                          d_out=[4096], seed=3, idx_kind="frac_neg", frac_neg=0.25),
         ]
     if n == 4:   # prefill, 8 sequences x 1024 tokens, one slot each
         seg = prefill_segments(4, 8, 1024, 8)
-        return [make_problem("prefill_sgmv", BF16, T=8192, D=4096, r=64, S=8,
+        return [make_problem("prefill_sgmv", dt(BF16), T=8192, D=4096, r=64, S=8,
                              d_out=[4096], seed=4, segments=seg)]
     if n == 5:   # large mixed batch, Zipf(1.1) popularity, 10% base-only, unsorted
-        return [make_problem("large_mixed", BF16, T=4096, D=8192, r=32, S=128,
+        return [make_problem("large_mixed", dt(BF16), T=4096, D=8192, r=32, S=128,
                              d_out=[8192], seed=5, idx_kind="zipf", frac_neg=0.10)]
     raise ValueError(n)
 

@@ -120,21 +120,28 @@ LORA_API lora_status lora_group(int T, int S, const int32_t* idx, void* meta, si
  *   x           device [T, ldx] (ldx >= D), dtype elements.
  *   A           host array of n_slices device pointers; A[i] is [S, r, D]
  *               contiguous (slot-major stack of rank-r down-projections).
+ *   idx         device int32 [T], this batch's adapter indices: the same
+ *               tensor (and contents) lora_group grouped into `meta`.
  *   buf         device fp32 [n_slices, T, r], fully overwritten.  The sums
  *               accumulate in fp32 and are stored in fp32 (pull 1804 names a
  *               half-precision intermediate as the accuracy problem).
  *   has_active  host flag: 0 means the caller knows no token has an adapter;
  *               the call then returns LORA_OK with nothing enqueued and buf
  *               untouched (pull 25914: no LoRA kernels, no zeroing).
- *   meta        the workspace lora_group filled from this batch's idx on this
- *               stream (or one ordered before it).
+ *   meta        the workspace lora_group filled from idx on this stream (or
+ *               one ordered before it).
+ * The grouping is checked against idx token by token: a token whose index
+ * differs from the group the workspace put it in (a workspace grouped from
+ * another batch) is not written, and the mismatch is counted, so that
+ * lora_check_errors returns LORA_ERR_BAD_INDEX; a stale grouping never yields
+ * a silently wrong row.
  * With r >= 16 and T >= 16 * S the slot groups of the grouping run on tcgen05
  * tensor cores (x rows gathered through the grouping permutation); otherwise
  * on CUDA cores.
  */
 LORA_API lora_status lora_shrink(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
-                        const void* x, int64_t ldx, const void* const* A, float* buf,
-                        int has_active, const void* meta, size_t meta_bytes,
+                        const void* x, int64_t ldx, const void* const* A, const int32_t* idx,
+                        float* buf, int has_active, const void* meta, size_t meta_bytes,
                         lora_stream_t stream);
 
 /*
@@ -152,6 +159,9 @@ LORA_API lora_status lora_shrink(lora_dtype dtype, int T, int D, int r, int S, i
  *   D_out             host int32 [n_slices], output width of each slice.
  *   scale             LoRA scaling factor (per-adapter scales: fold into B).
  *   y                 device [T, ldy] dtype, updated in place.
+ *   idx               device int32 [T], as for lora_shrink (checked against
+ *                     the grouping the same way: a mismatched row of y is not
+ *                     written, and is counted).
  *   y_col_off         host int64 [n_slices], first column of each slice in y;
  *                     slices must not overlap.
  *   has_active, meta  as for lora_shrink.
@@ -159,8 +169,8 @@ LORA_API lora_status lora_shrink(lora_dtype dtype, int T, int D, int r, int S, i
  */
 LORA_API lora_status lora_expand(lora_dtype dtype, int T, int r, int S, int n_slices,
                         const float* buf, int64_t buf_slice_stride, const void* const* B,
-                        const int32_t* D_out, float scale, void* y, int64_t ldy,
-                        const int64_t* y_col_off, int has_active, const void* meta,
+                        const int32_t* D_out, const int32_t* idx, float scale, void* y,
+                        int64_t ldy, const int64_t* y_col_off, int has_active, const void* meta,
                         size_t meta_bytes, lora_stream_t stream);
 
 /*
@@ -275,6 +285,13 @@ LORA_API const char* lora_status_string(lora_status status);
 
 /* Build identification: "liblora_b200 sm_100a <version>". */
 LORA_API const char* lora_build_info(void);
+
+/* Kernel launches this library has made in this process (all devices and
+ * streams), counting a launch recorded into a stream capture once; a graph
+ * replay launches nothing through the library and adds nothing.  For
+ * instrumentation: the difference across a call is the number of kernels
+ * that call enqueued. */
+LORA_API unsigned long long lora_launch_count(void);
 
 #ifdef __cplusplus
 }

@@ -49,7 +49,7 @@ class Dev:
             ops.shrink_segment(self.x, self.A, self.ss, self.sa, self.buf, self.meta)
         else:
             ops.group(self.idx, p.S, self.meta)
-            ops.shrink(self.x, self.A, self.buf, self.meta)
+            ops.shrink(self.x, self.A, self.idx, self.buf, self.meta)
         return self.buf
 
     def expand(self, buf=None, path=None):
@@ -61,7 +61,7 @@ class Dev:
             ops.expand_segment(b, self.B, self.ss, self.sa, self.y, self.meta, p.scale,
                                y_col_off=p.col_off)
         else:
-            ops.expand(b, self.B, self.y, self.meta, p.scale, y_col_off=p.col_off)
+            ops.expand(b, self.B, self.idx, self.y, self.meta, p.scale, y_col_off=p.col_off)
         return self.y
 
 

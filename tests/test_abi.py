@@ -70,10 +70,10 @@ FAKE = 0x10000  # a 16-byte aligned non-null address; never dereferenced
 
 
 def _shrink(L, dt=0, T=16, D=64, r=16, S=4, n=1, x=FAKE, ldx=64, A=(FAKE,), buf=FAKE, meta=FAKE,
-            meta_bytes=None):
+            meta_bytes=None, idx=FAKE):
     arr = (ctypes.c_void_p * max(len(A), 1))(*A)
     mb = L.lora_workspace_bytes(T, S) if meta_bytes is None else meta_bytes
-    return L.lora_shrink(dt, T, D, r, S, n, x, ldx, arr, buf, 1, meta, mb, None)
+    return L.lora_shrink(dt, T, D, r, S, n, x, ldx, arr, idx, buf, 1, meta, mb, None)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -93,19 +93,20 @@ def _shrink(L, dt=0, T=16, D=64, r=16, S=4, n=1, x=FAKE, ldx=64, A=(FAKE,), buf=
     (dict(x=0), _lib.LORA_ERR_INVALID_ARG),
     (dict(meta=0), _lib.LORA_ERR_INVALID_ARG),
     (dict(meta_bytes=64), _lib.LORA_ERR_INVALID_ARG),
+    (dict(idx=0), _lib.LORA_ERR_INVALID_ARG),                # the batch's indices are required
 ])
 def test_shrink_host_validation(L, kw, status):
     assert _shrink(L, **kw) == status
 
 
 def _expand(L, T=16, r=16, S=4, B=(FAKE, FAKE), d_out=(64, 32), off=(0, 64), ldy=96,
-            stride=16 * 16, buf=FAKE, y=FAKE):
+            stride=16 * 16, buf=FAKE, y=FAKE, idx=FAKE):
     n = len(B)
     arr = (ctypes.c_void_p * n)(*B)
     do = (ctypes.c_int32 * n)(*d_out)
     of = (ctypes.c_int64 * n)(*off)
-    return L.lora_expand(0, T, r, S, n, buf, stride, arr, do, ctypes.c_float(1.0), y, ldy, of, 1,
-                         FAKE, L.lora_workspace_bytes(T, S), None)
+    return L.lora_expand(0, T, r, S, n, buf, stride, arr, do, idx, ctypes.c_float(1.0), y, ldy,
+                         of, 1, FAKE, L.lora_workspace_bytes(T, S), None)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -117,6 +118,7 @@ def _expand(L, T=16, r=16, S=4, B=(FAKE, FAKE), d_out=(64, 32), off=(0, 64), ldy
     (dict(stride=258), _lib.LORA_ERR_MISALIGNED),
     (dict(y=FAKE + 4), _lib.LORA_ERR_MISALIGNED),
     (dict(B=(FAKE, 0)), _lib.LORA_ERR_INVALID_ARG),
+    (dict(idx=0), _lib.LORA_ERR_INVALID_ARG),
 ])
 def test_expand_host_validation(L, kw, status):
     assert _expand(L, **kw) == status
@@ -140,3 +142,24 @@ def test_group_host_validation(L):
     assert L.lora_group(16, 4, 0, FAKE, 4096, None) == _lib.LORA_ERR_INVALID_ARG
     assert L.lora_group(16, 4, FAKE, FAKE + 4, 4096, None) == _lib.LORA_ERR_MISALIGNED
     assert L.lora_group(16, 4, FAKE, FAKE, 16, None) == _lib.LORA_ERR_INVALID_ARG
+
+
+def test_launch_count_starts_at_zero_without_launches(L):
+    # nothing in this process has launched a kernel: the counter only moves
+    # on successful launches, and host-side rejections launch nothing
+    before = L.lora_launch_count()
+    assert _shrink(L, r=12) == _lib.LORA_ERR_UNSUPPORTED
+    assert L.lora_launch_count() == before == 0
+
+
+def test_has_active_from_host_indices():
+    import numpy as np
+    import torch
+    from gather_matmul_b200 import ops
+    assert not ops.active_from_host(np.array([-1, -1, 4, -7]), 4)   # 4 is outside [0, 4)
+    assert ops.active_from_host(np.array([-1, 3]), 4)
+    assert not ops.active_from_host(torch.full((5,), -1, dtype=torch.int32), 2)
+    assert not ops.active_from_host(np.array([], dtype=np.int32), 2)
+    assert ops._active(None, None, 4) == 1          # no host copy: the device decides
+    assert ops._active(None, np.array([-1]), 4) == 0
+    assert ops._active(False, np.array([0]), 4) == 0   # an explicit flag wins

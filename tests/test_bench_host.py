@@ -46,7 +46,37 @@ def test_workload_bytes_are_positive_and_consistent(n):
     for p in W.config(n):
         by = bench.algorithmic_bytes(p)
         assert by["step"] == by["shrink"] + by["expand"] + by["group"] > 0
-        assert bench.kernel_bytes(p, "fused") == by["shrink"] + by["expand"]
+        assert bench.call_bytes(p, "fused") == by["shrink"] + by["expand"]
+
+
+def test_kernel_names_follow_the_dispatch_rules():
+    # decode q_proj: T = 256 < 16 * 32 -> CUDA-core item kernels when not fused
+    p2 = W.config(2)[0]
+    assert bench.kernels_of(p2, "shrink", False) == ["shrink_items_kernel"]
+    assert bench.kernel_calls(p2, True) == ["fused"]
+    assert bench.kernels_of(p2, "fused", True) == ["bgmv_fused_kernel"]
+    # large mixed: r = 32, T = 4096 >= 16 * 128 -> grouped tensor-core kernels
+    p5 = W.config(5)[0]
+    assert bench.grouped_tc(p5)
+    assert bench.kernel_calls(p5, False) == ["group", "shrink", "expand"]
+    assert bench.kernels_of(p5, "expand", False) == ["sgmv_expand_tc_kernel"]
+    # prefill segments on tensor cores; rank 8 segments on the item kernels
+    p4 = W.config(4)[0]
+    assert bench.kernels_of(p4, "shrink", False) == ["sgmv_shrink_tc_kernel"]
+    q = W.make_problem("s", W.F16, T=64, D=64, r=8, S=2, d_out=[64], seed=1,
+                       segments=(np.array([0, 30, 64]), np.array([0, 1])))
+    assert bench.kernels_of(q, "expand", False) == ["segment_items_kernel", "expand_items_kernel"]
+
+
+def test_call_flops_and_e2e_window():
+    p = W.config(2)[0]
+    assert bench.call_flops(p, "fused") == bench.algorithmic_flops(p)
+    assert bench.call_flops(p, "shrink") + bench.call_flops(p, "expand") == \
+        bench.algorithmic_flops(p)
+    # at least K steps, and at least 100 ms at the estimated step time
+    assert bench.e2e_steps_for(1e-3, 20) == 100
+    assert bench.e2e_steps_for(1e-1, 20) == 20
+    assert bench.e2e_steps_for(1e-9, 20) == 20000      # capped
 
 
 def test_rotation_sets_cover_three_l2():

@@ -33,8 +33,8 @@ def test_no_active_launches_nothing_and_writes_nothing():
     torch.cuda.synchronize()
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
-        ops.shrink(d.x, d.A, d.buf, d.meta, has_active=False)
-        ops.expand(d.buf, d.B, d.y, d.meta, p.scale, has_active=False)
+        ops.shrink(d.x, d.A, d.idx, d.buf, d.meta, has_active=False)
+        ops.expand(d.buf, d.B, d.idx, d.y, d.meta, p.scale, has_active=False)
     # a call with has_active=0 enqueues nothing: the stream has no pending work
     assert s.query()
     torch.cuda.synchronize()
@@ -130,6 +130,45 @@ def test_bad_indices_are_flagged_and_treated_as_none():
     assert np.array_equal(host_bits(d.y)[[3, 17]], p.y[[3, 17]])
 
 
+@pytest.mark.parametrize("T,S,r", [(70, 5, 16), (400, 6, 32)],
+                         ids=["cuda-core-items", "tensor-core-grouped"])
+def test_stale_grouping_is_flagged_never_silently_wrong(T, S, r):
+    # The workspace is grouped from batch k's indices, then the compute calls
+    # get batch k+1 (same sizes, a third of the tokens on another slot or
+    # none).  Every token whose index changed must be left unwritten (buf
+    # keeps its NaN sentinel, y its input bits) and counted; every other row
+    # must still be right.
+    import dataclasses
+    pk = _p(seed=50, T=T, S=S, r=r, D=1032, d_out=(256, 64), kind="uniform_neg")
+    rng = np.random.default_rng(51)
+    idx2 = pk.idx.copy()
+    moved = rng.choice(T, size=T // 3, replace=False)
+    shift = 1 + rng.integers(0, S, size=moved.size)          # never a multiple of S + 1
+    idx2[moved] = (idx2[moved] + 1 + shift) % (S + 1) - 1
+    assert np.all(idx2[moved] != pk.idx[moved])
+    q = dataclasses.replace(pk, idx=idx2.astype(np.int32))
+    d = Dev(q)
+    ops.group(torch.from_numpy(pk.idx).cuda(), S, d.meta)     # batch k's grouping
+    ops.shrink(d.x, d.A, d.idx, d.buf, d.meta)                # batch k+1's data
+    ops.expand(d.buf, d.B, d.idx, d.y, d.meta, q.scale, y_col_off=q.col_off)
+    assert ops.check_errors(d.meta) == _lib.LORA_ERR_BAD_INDEX
+    keep = np.ones(T, dtype=bool)
+    keep[moved] = False
+    g = d.buf.detach().cpu().double().numpy()
+    assert np.all(np.isnan(g[:, moved])), "a row of a moved token was written"
+    assert np.array_equal(host_bits(d.y)[moved], q.y[moved]), "y of a moved token changed"
+    buf_ref, cabs = oracle_shrink(q)
+    assert_buf_close(torch.from_numpy(g[:, keep]), buf_ref[:, keep], cabs[:, keep])
+    y_ref = oracle_expand(q, buf_ref)
+    gy = oracle.decode(q.dtype, host_bits(d.y))
+    assert np.all(np.abs(gy[keep] - y_ref[keep]) <= 1e-2 * (1 + np.abs(y_ref[keep])))
+    # grouped from the right batch, the same calls are clean
+    d2 = Dev(q)
+    d2.shrink()
+    d2.expand()
+    assert ops.check_errors(d2.meta) == _lib.LORA_OK
+
+
 def test_malformed_segments_are_flagged():
     p = W.make_problem("s", W.BF16, T=64, D=256, r=16, S=3, d_out=[64], seed=1,
                        segments=(np.array([0, 40, 30, 64]), np.array([0, 1, 2])))
@@ -165,6 +204,28 @@ def test_integer_inputs_match_oracle_bitwise(dt, D, r):
         assert np.array_equal(buf.cpu().double().numpy(), buf_ref)
         y_ref = oracle_expand(p, buf_ref)
         assert np.array_equal(oracle.decode(p.dtype, host_bits(y)), y_ref)
+
+
+@pytest.mark.parametrize("dt,D,T,S", [(W.F16, 64, 200, 3), (W.F16, 64, 300, 2),
+                                      (W.BF16, 8, 200, 3), (W.BF16, 8, 300, 2)],
+                         ids=["f16-small-groups", "f16-full-tiles", "bf16-small-groups",
+                              "bf16-full-tiles"])
+def test_integer_inputs_grouped_tensor_cores_bitwise(dt, D, T, S):
+    # T >= 16 S with r = 16: the per-token batch runs through the grouping on
+    # the tcgen05 kernels (groups of about 50 rows take the operand-swapped
+    # expand, about 100 rows the full 128-row tile).  x, A, B in {-1,0,1},
+    # y in [-8,8]: |buf| <= D and |y| <= 8 + 16 D stay exact (fp16: <= 1032
+    # < 2048; bf16: <= 136 < 256), through the hi + lo split as well, so the
+    # GPU equals the oracle bit for bit.
+    p = W.make_problem("int_tc", dt, T=T, D=D, r=16, S=S, d_out=[136, 64], scale=1.0,
+                       seed=T + S, idx_kind="uniform_neg", values="int")
+    d = Dev(p)
+    buf_ref, _ = oracle_shrink(p)
+    buf = d.shrink()
+    y = d.expand()
+    torch.cuda.synchronize()
+    assert np.array_equal(buf.cpu().double().numpy(), buf_ref)
+    assert np.array_equal(oracle.decode(p.dtype, host_bits(y)), oracle_expand(p, buf_ref))
 
 
 def test_sgmv_equals_bgmv_on_expanded_indices():
@@ -205,8 +266,8 @@ def test_stream_and_graph_capture():
     torch.cuda.synchronize()
     with torch.cuda.graph(g, stream=s):
         ops.group(d.idx, p.S, d.meta)
-        ops.shrink(d.x, d.A, d.buf, d.meta)
-        ops.expand(d.buf, d.B, d.y, d.meta, p.scale)
+        ops.shrink(d.x, d.A, d.idx, d.buf, d.meta)
+        ops.expand(d.buf, d.B, d.idx, d.y, d.meta, p.scale)
     d.y.copy_(y_in)
     g.replay()
     torch.cuda.synchronize()
@@ -239,7 +300,7 @@ def test_power_of_two_scale_scales_y_exactly(path):
             if p.segmented:
                 ops.expand_segment(b, d.B, d.ss, d.sa, d.y, d.meta, scale, y_col_off=p.col_off)
             else:
-                ops.expand(b, d.B, d.y, d.meta, scale, y_col_off=p.col_off)
+                ops.expand(b, d.B, d.idx, d.y, d.meta, scale, y_col_off=p.col_off)
         torch.cuda.synchronize()
         ys.append(oracle.decode(p.dtype, host_bits(d.y)))
     assert np.any(ys[0] != 0)

@@ -48,6 +48,16 @@ def test_config_full_size(cfg, proj):
     _run_and_check(p)
 
 
+@pytest.mark.parametrize("cfg", [4, 5], ids=["cfg4-prefill-f16", "cfg5-large-mixed-f16"])
+def test_tensor_core_workloads_full_size_fp16(cfg):
+    """The two workloads that run on the tcgen05 kernels (prefill segments and
+    the large mixed per-token batch through the grouping), drawn in fp16: the
+    fp16 instruction descriptors, the fp16 hi + lo split of the intermediate
+    and fp16 rounding of y, at full size."""
+    p = W.config(cfg, dtype=W.F16)[0]
+    _run_and_check(p)
+
+
 SHAPES = [
     # dtype, T, D, r, S, d_out, idx_kind, shared_A
     (W.F16, 1, 8, 8, 1, [8], "uniform", False),
