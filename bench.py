@@ -649,7 +649,56 @@ def configs_block(stream, peak, tf_peak, reps=256):
                              "tokens_per_s": round(layer[0][2] / t3, 1),
                              "gbs": round(b3 / t3 / 1e9, 1),
                              "frac_hbm": round(b3 / t3 / 1e9 / peak, 4)}
+    out["cfg3:layer_one_grouping"] = layer_one_grouping(stream, peak, reps)
     return out
+
+
+def layer_one_grouping(stream, peak, reps):
+    """The three fused-slice projections of one decoder layer as a decode
+    step runs them: the batch's grouping built once (lora_group) and shared by
+    every projection's shrink and expand (the projections of one batch carry
+    the same indices)."""
+    from gather_matmul_b200 import ops
+    probs = W.config(3)
+    sets = [make_sets(p) for p in probs]
+    n = min(len(s) for s in sets)
+
+    def one(k):
+        d0 = sets[0][k % n]
+        ops.group(d0.idx, probs[0].S, d0.meta)
+        for p, ss in zip(probs, sets):
+            d = ss[k % n]
+            ops.shrink(d.x, d.A, d0.idx, d.buf, d0.meta)
+            ops.expand(d.buf, d.B, d0.idx, d.y, d0.meta, p.scale, y_col_off=p.col_off)
+
+    graphs = []
+    G = 32
+    for start in range(0, reps, G):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for k in range(start, min(reps, start + G)):
+                one(k)
+        graphs.append(g)
+
+    def run():
+        with torch.cuda.stream(stream):
+            for g in graphs:
+                g.replay()
+    run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / reps
+    by = algorithmic_bytes(probs[0])["group"] + sum(
+        algorithmic_bytes(p, with_group=False)["step"] for p in probs)
+    del graphs, sets
+    torch.cuda.empty_cache()
+    return {"us_per_layer": round(t * 1e6, 3), "tokens_per_s": round(probs[0].T / t, 1),
+            "gbs": round(by / t / 1e9, 1), "frac_hbm": round(by / t / 1e9 / peak, 4),
+            "launches_per_layer": 1 + 2 * len(probs)}
 
 
 def idle_call_us(calls=2000):
@@ -683,6 +732,138 @@ def idle_call_us(calls=2000):
     for _ in range(calls):
         fn(*args)
     out["c_abi"] = round((time.perf_counter() - t0) / calls * 1e6, 3)
+    return out
+
+
+def graph_specialization(stream, reps=200, T=256, S=32, r=16):
+    """LoRA enabled but idle, with one graph set and with graphs specialised
+    on has_lora ("[LoRA] LoRA cuda graph specialization": two graph sets,
+    dispatch on the batch's flag; its latency logs: 10.5 % -> 1.4 %).
+
+    Stand-in for one decoder layer of a decode step at Llama-3-8B shapes:
+    the base projections qkv (4096 -> 4096+1024+1024), o (4096 -> 4096),
+    gate_up (4096 -> 14336+14336) and down (14336 -> 4096) as torch matmuls
+    (the base model, not this library), each followed by its LoRA update
+    through lora_bgmv; T tokens, S slots, rank r, bf16, random weights.
+    Device times per step from CUDA events around `reps` graph replays."""
+    from gather_matmul_b200 import ops
+    from gather_matmul_b200.graphs import LoraGraphSet
+    g = torch.Generator(device="cuda").manual_seed(80)
+    td = torch.bfloat16
+    rnd = lambda *shape, std=1.0: (torch.randn(*shape, generator=g, device="cuda") * std).to(td)
+    projs = [(4096, [4096, 1024, 1024]), (4096, [4096]), (4096, [14336, 14336]), (14336, [4096])]
+    layers = []
+    for D, d_out in projs:
+        n = sum(d_out)
+        layers.append(dict(
+            D=D, d_out=d_out, off=list(np.concatenate([[0], np.cumsum(d_out)[:-1]]).astype(int)),
+            x=rnd(T, D), W=rnd(n, D, std=0.02), y=torch.empty(T, n, dtype=td, device="cuda"),
+            A=[rnd(S, r, D, std=0.02) for _ in d_out], B=[rnd(S, o, r, std=0.02) for o in d_out],
+            buf=torch.empty(len(d_out), T, r, dtype=torch.float32, device="cuda"),
+            meta=ops.workspace(T, S)))
+    idx = torch.empty(T, dtype=torch.int32, device="cuda")
+    rng = np.random.default_rng(81)
+    idx_active = rng.integers(0, S, size=T).astype(np.int32)
+    idx_idle = np.full(T, -1, dtype=np.int32)
+
+    def step(has_lora):
+        for L in layers:
+            torch.matmul(L["x"], L["W"].t(), out=L["y"])
+            if has_lora:
+                ops.bgmv(L["x"], L["A"], L["B"], idx, L["y"], L["buf"], L["meta"], 1.0,
+                         y_col_off=L["off"])
+
+    idx.copy_(torch.from_numpy(idx_active))
+    gs = LoraGraphSet(step, stream).capture()
+
+    def timed(body):
+        for _ in range(3):
+            body()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            body()
+        host = time.perf_counter() - t0
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 1e3 / reps, host / reps
+
+    with torch.cuda.stream(stream):
+        t_base, _ = timed(lambda: gs.replay(False))
+        idx.copy_(torch.from_numpy(idx_idle))
+        t_idle_one, _ = timed(lambda: gs.replay(True))
+        t_idle_spec, host_spec = timed(lambda: gs.replay_for(idx_idle, S))
+        idx.copy_(torch.from_numpy(idx_active))
+        t_active, _ = timed(lambda: gs.replay_for(idx_active, S))
+    t0 = time.perf_counter()
+    for _ in range(1000):
+        ops.active_from_host(idx_idle, S)
+    decide = (time.perf_counter() - t0) / 1000
+    launches = {"without_lora": gs.lora_launches[False], "with_lora": gs.lora_launches[True]}
+    del gs
+    return {
+        "stand_in": f"decode layer, T={T}, Llama-3-8B qkv/o/gate_up/down base matmuls + "
+                    f"lora_bgmv per projection, S={S} r={r} bf16",
+        "us_base_graph": round(t_base * 1e6, 2),
+        "us_idle_one_graph_set": round(t_idle_one * 1e6, 2),
+        "us_idle_specialized": round(t_idle_spec * 1e6, 2),
+        "us_lora_active": round(t_active * 1e6, 2),
+        "overhead_idle_one_graph_set": round(t_idle_one / t_base - 1, 4),
+        "overhead_idle_specialized": round(t_idle_spec / t_base - 1, 4),
+        "host_us_per_dispatch": round(host_spec * 1e6, 2),
+        "host_us_has_lora_from_indices": round(decide * 1e6, 2),
+        "library_launches_per_step": launches,
+    }
+
+
+def laning_block(stream, peak, reps=256):
+    """The laned shrink (every slot's A as one [S*r, D] matrix on tensor
+    cores, each token keeping its own lanes, no grouping) against the grouped
+    shrink (group-by-slot, then the shrink over the grouping), on the
+    small-rank per-token workloads.  Same algorithmic bytes, so the HBM
+    fractions compare directly."""
+    from gather_matmul_b200 import ops
+    out = {}
+    for n in (1, 2):
+        p = W.config(n)[0]
+        sets = make_sets(p)
+        res = {}
+        calls = {
+            "laned_shrink": lambda d: ops.shrink_laned(d.x, d.A, d.idx, d.buf, d.meta),
+            "group_then_shrink": lambda d: (ops.group(d.idx, p.S, d.meta),
+                                            ops.shrink(d.x, d.A, d.idx, d.buf, d.meta)),
+        }
+        for name, fn in calls.items():
+            graphs = []
+            for start in range(0, reps, 64):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for k in range(start, min(reps, start + 64)):
+                        fn(sets[k % len(sets)])
+                graphs.append(g)
+            with torch.cuda.stream(stream):
+                for g in graphs:
+                    g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            with torch.cuda.stream(stream):
+                for g in graphs:
+                    g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1) / 1e3 / reps
+            by = algorithmic_bytes(p)["shrink"] + (algorithmic_bytes(p)["group"]
+                                                   if name == "group_then_shrink" else 0)
+            res[name] = {"us": round(t * 1e6, 3), "gbs": round(by / t / 1e9, 1),
+                         "frac_hbm": round(by / t / 1e9 / peak, 4)}
+            del graphs
+        res["lane_flops_per_useful"] = p.S
+        out[f"cfg{n}:{p.name}"] = res
+        del sets
+        torch.cuda.empty_cache()
     return out
 
 
@@ -775,6 +956,8 @@ def run_ours(args):
     if blocks is not None:
         blocks["idle_call_us"] = idle_call_us()
         line["configs"] = blocks
+        line["graph_specialization"] = graph_specialization(stream)
+        line["laning"] = laning_block(stream, peak)
     print(json.dumps(line), flush=True)
     barrier(ws)
 

@@ -43,6 +43,9 @@ SIGNATURES = {
     "lora_check_errors": (_i32, [_vp, _sz, _vp]),
     "lora_shrink_noalloc": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp,
                                    _vp, _i32, _vp]),
+    "lora_shrink_laned": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp,
+                                 _i32, _vp, _sz, _vp]),
+    "lora_set_slot_ranks": (_i32, [_i32, _vp, _vp, _sz, _vp]),
     "lora_status_string": (ctypes.c_char_p, [_i32]),
     "lora_build_info": (ctypes.c_char_p, []),
     "lora_launch_count": (ctypes.c_ulonglong, []),

@@ -52,9 +52,12 @@ def build(force=False, verbose=False, out=LIB, extra=()):
             print(" ".join(cmd))
         subprocess.run(cmd, check=True)
         objs.append(obj)
+    # link to a temporary name, then rename: a reader never sees a partial file
+    tmp = out + ".tmp"
     cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static",
-           "-Xcompiler", "-fPIC", "-o", out, *objs]
+           "-Xcompiler", "-fPIC", "-o", tmp, *objs]
     subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
     return out
 
 

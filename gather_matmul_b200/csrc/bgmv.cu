@@ -115,7 +115,9 @@ shrink_items_kernel(const ShrinkArgs a) {
       (&sacc[0][0][0])[e] = 0.f;
     __syncthreads();
 
-    if (slot < 0) {          // tokens without an adapter: buf rows are zero
+    // tokens without an adapter, and rank groups past the slot's own rank:
+    // zero buf columns, nothing read
+    if (slot < 0 || j0 >= slot_rank(a.meta, a.S, slot, r)) {
       if (crank == 0)
         for (int e = tid; e < nt * kJR; e += kThreads)
           if (stok[e / kJR] >= 0) bufs[(size_t)stok[e / kJR] * r + j0 + e % kJR] = 0.f;
@@ -246,14 +248,16 @@ expand_items_kernel(const ExpandArgs a) {
     __syncthreads();
     if (!active) continue;
 
-    // this thread's CPL rows of B_i[slot], r values each, as fp32
+    // this thread's CPL rows of B_i[slot], the slot's own rank k of its r
+    // values each (the padding past k is neither read nor multiplied), as fp32
+    const int kslot = slot_rank(a.meta, a.S, slot, R);
     float bf[CPL][R];
     const E* Bg = static_cast<const E*>(a.B[slice]) + ((size_t)slot * a.D_out[slice] + o0) * R;
 #pragma unroll
     for (int c = 0; c < CPL; ++c)
 #pragma unroll
       for (int j8 = 0; j8 < R / 8; ++j8) {
-        uint4 u = ldg_stream(Bg + c * R + j8 * 8);
+        uint4 u = j8 * 8 < kslot ? ldg_stream(Bg + c * R + j8 * 8) : make_uint4(0, 0, 0, 0);
         Elem<E>::to_f32(u, &bf[c][j8 * 8]);
       }
 
@@ -273,6 +277,7 @@ expand_items_kernel(const ExpandArgs a) {
         for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
 #pragma unroll
         for (int j4 = 0; j4 < R / 4; ++j4) {
+          if (j4 * 4 >= kslot) break;
           const float4 bv = *reinterpret_cast<const float4*>(&sbuf[k][j4 * 4]);
 #pragma unroll
           for (int c = 0; c < CPL; ++c) {

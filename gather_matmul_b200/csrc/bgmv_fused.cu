@@ -178,9 +178,10 @@ bgmv_fused_kernel(const __grid_constant__ FusedParams P) {
 
   // Copies are issued in the order they are needed: the slot's A rows and the
   // first chunk's x rows feed the shrink, B and y only the expand.  When the
-  // batch has at least two tokens per slot on average the A rows are fetched
-  // before the index scan, on the guess that this slot has tokens; a CTA whose
-  // slot turns out empty waits for them before it exits.
+  // batch has at least two tokens per slot on average the slot's A rows and B
+  // tiles (they depend on the slot alone) are fetched before the index scan,
+  // on the guess that this slot has tokens; a CTA whose slot turns out empty
+  // waits for them before it exits.
   const bool spec_A = a.T >= 2 * a.S;
   auto issue_A = [&]() {
     if (lane == 0) {
@@ -191,11 +192,24 @@ bgmv_fused_kernel(const __grid_constant__ FusedParams P) {
           ptx::bulk_g2s(sA + (size_t)j * L.pitchA, Ag + (size_t)j * D, dn * 2, barA);
     }
   };
+  auto issue_B = [&]() {
+    if (lane == 0) {
+      const int nbox = (on + kBoxRows - 1) / kBoxRows;
+      const int nB = (nbox - warp + kFWarps - 1) / kFWarps;
+      ptx::mbar_arrive_expect_tx(barB, (uint32_t)(max(nB, 0) * L.boxBytes));
+      for (int b = warp; b < nbox; b += kFWarps)
+        ptx::tma_load_2d(sB + (size_t)b * L.boxBytes, &P.tmB[slice], 0,
+                         g * Dout + o0 + b * kBoxRows, barB);
+    }
+  };
   if (!a.pdl_early) ptx::grid_dep_wait();
   // the first block of indices is requested ahead of the A rows, so that the
   // scan does not queue behind them; each block prefetches the next
   int v_next = tid < a.T ? a.idx[tid] : -1;
-  if (spec_A) issue_A();
+  if (spec_A) {
+    issue_A();
+    issue_B();
+  }
 
   // 1. this slot's tokens, in token order
   int n_tok = 0;
@@ -240,7 +254,10 @@ bgmv_fused_kernel(const __grid_constant__ FusedParams P) {
   }
   ptx::grid_dep_launch_dependents();
   if (n_tok == 0) {                 // the same for every CTA of the cluster
-    if (spec_A && tid == 0) ptx::mbar_wait(barA, 0);   // the A rows fetched on a guess
+    if (spec_A && tid == 0) {         // the A rows and B tiles fetched on a guess
+      ptx::mbar_wait(barA, 0);
+      ptx::mbar_wait(barB, 0);
+    }
     return;
   }
 
@@ -271,14 +288,7 @@ bgmv_fused_kernel(const __grid_constant__ FusedParams P) {
   // 2. the first chunk's x rows, the slot's B rows (output chunk), the first
   // chunk's y rows; lane 0 of every warp issues its share
   issue_x(0, min(kTB, n_tok));
-  if (lane == 0) {
-    const int nbox = (on + kBoxRows - 1) / kBoxRows;
-    const int nB = (nbox - warp + kFWarps - 1) / kFWarps;
-    ptx::mbar_arrive_expect_tx(barB, (uint32_t)(max(nB, 0) * L.boxBytes));
-    for (int b = warp; b < nbox; b += kFWarps)
-      ptx::tma_load_2d(sB + (size_t)b * L.boxBytes, &P.tmB[slice], 0,
-                       g * Dout + o0 + b * kBoxRows, barB);
-  }
+  if (!spec_A) issue_B();
   issue_y(0, min(kTB, n_tok));
 
   int phase = 0;

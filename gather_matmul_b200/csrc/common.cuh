@@ -19,35 +19,54 @@ constexpr int kMaxRank = 64;
 //   slot_off       int32 [S + 2]: slot g's tokens are perm[slot_off[g] ..
 //                  slot_off[g+1]); [slot_off[S], slot_off[S+1]) = the tokens
 //                  without an adapter
+//   slot_rank      int32 [S]: each slot's own rank (lora_set_slot_ranks),
+//                  used when the header's has_ranks is set
 //   perm           int32 [T]
 //   items          int4 [max_items]: {slot (-1 = none), begin, end, flags}
+//   hist           int32 [group_ctas(T)][S + 1]: per-CTA slot counts of the
+//                  grouping kernel
 // ---------------------------------------------------------------------------
 struct MetaHeader {
   int bad_index;      // count of indices outside [-1, S) (accumulates)
-  int bad_meta;       // malformed segment lists, or metadata built for other
-                      // sizes than the call's (accumulates)
+  int bad_meta;       // malformed segment lists, metadata built for other
+                      // sizes than the call's, rows whose index disagrees
+                      // with the grouping, timed-out waits (accumulates)
   int n_items;        // items in the work list
   int n_active;       // tokens with an adapter
   int T, S;           // sizes the metadata was built for
-  int pad[58];
+  int bar_count;      // grouping kernel's inter-CTA barrier: CTAs arrived
+  int bar_gen;        //   and completed barrier generations
+  int has_ranks;      // slot_rank holds per-slot ranks
+  int pad[55];
 };
 static_assert(sizeof(MetaHeader) == 256, "header is 256 bytes");
+
+// CTAs of the grouping kernel for T tokens: one per 2048 tokens, at most 64
+// (all resident at once, so they can meet at a barrier).
+constexpr int kGroupChunkMin = 2048;
+constexpr int kGroupMaxCtas = 64;
+__host__ __device__ inline int group_ctas(int T) {
+  const int nb = (T + kGroupChunkMin - 1) / kGroupChunkMin;
+  return nb < 1 ? 1 : (nb > kGroupMaxCtas ? kGroupMaxCtas : nb);
+}
 
 enum ItemFlags { kItemDirect = 1 };   // token = position (segments), no perm
 
 struct MetaLayout {
-  size_t off_slot, off_perm, off_items, total;
+  size_t off_slot, off_rank, off_perm, off_items, off_hist, total;
   int max_items;
   __host__ __device__ static size_t a256(size_t v) { return (v + 255) & ~size_t(255); }
   __host__ __device__ MetaLayout(int T, int S) {
     int tt = T > 0 ? T : 1;
     off_slot = 256;
-    off_perm = off_slot + a256(sizeof(int) * (size_t)(S + 2));
+    off_rank = off_slot + a256(sizeof(int) * (size_t)(S + 2));
+    off_perm = off_rank + a256(sizeof(int) * (size_t)S);
     off_items = off_perm + a256(sizeof(int) * (size_t)tt);
     // per-token grouping: <= T/16 + (S + 1) items; segments: <= T/16 + n_seg
     // with n_seg <= T + 1.
     max_items = T / kItemTokens + (S + 1 > T + 1 ? S + 1 : T + 1) + 2;
-    total = off_items + a256(sizeof(int4) * (size_t)max_items);
+    off_hist = off_items + a256(sizeof(int4) * (size_t)max_items);
+    total = off_hist + a256(sizeof(int) * (size_t)group_ctas(T) * (size_t)(S + 1));
   }
 };
 
@@ -130,6 +149,18 @@ __device__ __forceinline__ int checked_items(const char* meta, int T, int S) {
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
     atomicAdd(const_cast<int*>(&h->bad_meta), 1);
   return 0;
+}
+
+// Rank slot g really uses, for a call of rank R: the slot's own rank from
+// lora_set_slot_ranks rounded up to a multiple of 8, or R when none is set
+// (or the value is outside (0, R)).  Rows of A and columns of B past it are
+// zero padding that the kernels neither read nor multiply.
+__device__ __forceinline__ int slot_rank(const char* meta, int S, int g, int R) {
+  const MetaHeader* h = reinterpret_cast<const MetaHeader*>(meta);
+  if (!h->has_ranks || g < 0 || g >= S) return R;
+  const int v = reinterpret_cast<const int*>(meta + MetaLayout::a256(256) +
+                                             MetaLayout::a256(sizeof(int) * (size_t)(S + 2)))[g];
+  return (v <= 0 || v >= R) ? R : ((v + 7) & ~7);
 }
 
 // Whether token `tok` really belongs to the group of a per-token grouping it

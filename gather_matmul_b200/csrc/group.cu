@@ -55,41 +55,96 @@ __device__ int block_exclusive_scan(int* a, int n, int* warp_tmp) {
   return total;
 }
 
-// One CTA.  Shared memory: cnt[kGroupWarps][K], tot[K], base[K], ni[K],
-// plus 65 ints of scan scratch, with K = S + 1 keys (slot S = no adapter).
+// Generation barrier of the grouping kernel's CTAs, kept in the workspace
+// header.  Thread 0 of each CTA calls it once its CTA's histogram row is
+// written and fenced.  The last CTA to arrive resets the count and opens the
+// next generation, so the barrier is reusable whatever the CTA count of the
+// next launch.  The wait is bounded (about one second): on a timeout it
+// returns false and the caller records an error instead of hanging.
+__device__ bool group_barrier(MetaHeader* hdr, int nb) {
+  volatile int* gen = &hdr->bar_gen;
+  const int g0 = *gen;
+  __threadfence();
+  if (atomicAdd(&hdr->bar_count, 1) == nb - 1) {
+    atomicExch(&hdr->bar_count, 0);
+    __threadfence();
+    atomicAdd(&hdr->bar_gen, 1);
+    return true;
+  }
+  uint64_t t0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  while (*gen == g0) {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (t - t0 > 1000000000ull) return false;
+    __nanosleep(200);
+  }
+  __threadfence();
+  return true;
+}
+
+constexpr int kLoadBatch = 8;   // indices a lane has in flight at once
+
+// group_ctas(T) CTAs, each over a contiguous chunk of the tokens; each warp
+// over a contiguous part of its CTA's chunk, so CTA, warp and lane order is
+// token order and the scatter is stable.  Shared memory: cnt[kGroupWarps][K],
+// tot[K], base[K], pre[K], ni[K] and 66 ints of scan scratch, K = S + 1 keys
+// (key S = no adapter).
+//   1. per-warp counts of each key (warp match_any), summed into this CTA's
+//      row of the workspace histogram;
+//   2. barrier over the CTAs;
+//   3. every CTA reads the histogram: each key's total and the part of it in
+//      earlier CTAs; block scans give each key's first position and the work
+//      list offsets;
+//   4. stable scatter of this CTA's tokens into perm; CTA 0 writes the slot
+//      offsets and header, the work items are shared out by key.
 __global__ void __launch_bounds__(kGroupThreads, 1)
 group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ meta) {
   extern __shared__ int smem[];
   const int K = S + 1;
   int* cnt = smem;                          // [warp][key]
-  int* tot = cnt + kGroupWarps * K;         // count per key
+  int* tot = cnt + kGroupWarps * K;         // this CTA's count, then the total, per key
   int* base = tot + K;                      // first position per key
-  int* ni = base + K;                       // items per key, then item offsets
-  int* scratch = ni + K;                    // 65 ints
+  int* pre = base + K;                      // tokens of the key in earlier CTAs
+  int* ni = pre + K;                        // items per key, then item offsets
+  int* scratch = ni + K;                    // 65 ints of scan scratch + a flag
 
   MetaLayout L(T, S);
   MetaHeader* hdr = reinterpret_cast<MetaHeader*>(meta);
   int* slot_off = reinterpret_cast<int*>(meta + L.off_slot);
   int* perm = reinterpret_cast<int*>(meta + L.off_perm);
   int4* items = reinterpret_cast<int4*>(meta + L.off_items);
+  int* hist = reinterpret_cast<int*>(meta + L.off_hist);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nb = gridDim.x, cta = blockIdx.x;
+  const int chunk = (T + nb - 1) / nb;
+  const int c0 = min(T, cta * chunk), c1 = min(T, c0 + chunk);
+  const int wchunk = (((c1 - c0) + kGroupWarps - 1) / kGroupWarps + 31) & ~31;
+  const int beg = min(c1, c0 + warp * wchunk);
+  const int end = min(c1, beg + wchunk);
+
   for (int i = tid; i < kGroupWarps * K; i += kGroupThreads) cnt[i] = 0;
   __syncthreads();
 
-  // Each warp owns one contiguous range of tokens, walked 32 at a time.
-  const int chunk = (((T + kGroupWarps - 1) / kGroupWarps) + 31) & ~31;
-  const int beg = warp * chunk;
-  const int end = min(T, beg + chunk);
   int bad = 0;
-  for (int b = beg; b < end; b += 32) {
-    int t = b + lane;
-    bool valid = t < end;
-    int v = valid ? idx[t] : -1;
-    if (valid && (v < -1 || v >= S)) ++bad;
-    int key = valid ? ((v >= 0 && v < S) ? v : S) : -1;
-    unsigned peers = __match_any_sync(0xffffffffu, key);
-    if (valid && lane == __ffs(peers) - 1) cnt[warp * K + key] += __popc(peers);
+  for (int b0 = beg; b0 < end; b0 += 32 * kLoadBatch) {
+    int v[kLoadBatch];
+#pragma unroll
+    for (int u = 0; u < kLoadBatch; ++u) {
+      const int t = b0 + 32 * u + lane;
+      v[u] = t < end ? __ldg(idx + t) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kLoadBatch; ++u) {
+      if (b0 + 32 * u >= end) break;              // warp-uniform
+      const int t = b0 + 32 * u + lane;
+      const bool valid = t < end;
+      if (valid && (v[u] < -1 || v[u] >= S)) ++bad;
+      const int key = valid ? ((v[u] >= 0 && v[u] < S) ? v[u] : S) : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, key);
+      if (valid && lane == __ffs(peers) - 1) cnt[warp * K + key] += __popc(peers);
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
@@ -97,34 +152,59 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
   __syncthreads();
 
   for (int k = tid; k < K; k += kGroupThreads) {
-    int s = 0;
-    for (int w = 0; w < kGroupWarps; ++w) s += cnt[w * K + k];
-    tot[k] = s;
-    base[k] = s;
-    ni[k] = (s + kItemTokens - 1) / kItemTokens;
+    int c = 0;
+    for (int w = 0; w < kGroupWarps; ++w) c += cnt[w * K + k];
+    tot[k] = c;
+    if (nb > 1) {
+      hist[cta * K + k] = c;
+      __threadfence();
+    }
+  }
+  __syncthreads();
+  if (nb > 1) {
+    if (tid == 0) scratch[65] = group_barrier(hdr, nb) ? 1 : 0;
+    __syncthreads();
+    if (!scratch[65]) {                           // another CTA never arrived
+      if (tid == 0) atomicAdd(&hdr->bad_meta, 1);
+      return;
+    }
+  }
+
+  for (int k = tid; k < K; k += kGroupThreads) {
+    int all = 0, before = 0;
+    for (int c = 0; c < nb; ++c) {
+      const int v = c == cta ? tot[k] : __ldcg(hist + c * K + k);
+      all += v;
+      before += c < cta ? v : 0;
+    }
+    tot[k] = all;
+    base[k] = all;
+    pre[k] = before;
+    ni[k] = (all + kItemTokens - 1) / kItemTokens;
   }
   __syncthreads();
   // K <= LORA_MAX_SLOTS + 1 <= 2 * kGroupThreads
   block_exclusive_scan(base, K, scratch);
-  int n_items = block_exclusive_scan(ni, K, scratch);
+  const int n_items = block_exclusive_scan(ni, K, scratch);
 
   for (int k = tid; k < K; k += kGroupThreads) {
-    slot_off[k] = base[k];
-    int run = base[k];
+    int run = base[k] + pre[k];
     for (int w = 0; w < kGroupWarps; ++w) {   // per-(warp, key) start positions
-      int c = cnt[w * K + k];
+      const int c = cnt[w * K + k];
       cnt[w * K + k] = run;
       run += c;
     }
-    int it0 = ni[k];
-    int n = tot[k];
-    for (int j = 0; j * kItemTokens < n; ++j) {
-      int b0 = base[k] + j * kItemTokens;
-      int e0 = min(base[k] + n, b0 + kItemTokens);
-      items[it0 + j] = make_int4(k < S ? k : -1, b0, e0, 0);
+    if (cta == 0) slot_off[k] = base[k];
+    if (k % nb == cta) {
+      const int it0 = ni[k], n = tot[k];
+      for (int j = 0; j * kItemTokens < n; ++j) {
+        const int b0 = base[k] + j * kItemTokens;
+        const int e0 = min(base[k] + n, b0 + kItemTokens);
+        items[it0 + j] = make_int4(k < S ? k : -1, b0, e0, 0);
+      }
     }
   }
-  if (tid == 0) {
+  if (cta == 0 && tid == 0) {
     slot_off[K] = T;
     hdr->n_items = n_items;
     hdr->n_active = base[S];
@@ -135,20 +215,29 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
 
   // Stable scatter: the same walk; a token's rank among equal keys of its
   // 32-token step comes from the match mask.
-  for (int b = beg; b < end; b += 32) {
-    int t = b + lane;
-    bool valid = t < end;
-    int v = valid ? idx[t] : -1;
-    int key = valid ? ((v >= 0 && v < S) ? v : S) : -1;
-    unsigned peers = __match_any_sync(0xffffffffu, key);
-    int pos = 0;
-    if (valid) pos = cnt[warp * K + key] + __popc(peers & lanemask_lt());
-    __syncwarp();
-    if (valid) {
-      perm[pos] = t;
-      if (lane == __ffs(peers) - 1) cnt[warp * K + key] += __popc(peers);
+  for (int b0 = beg; b0 < end; b0 += 32 * kLoadBatch) {
+    int v[kLoadBatch];
+#pragma unroll
+    for (int u = 0; u < kLoadBatch; ++u) {
+      const int t = b0 + 32 * u + lane;
+      v[u] = t < end ? __ldg(idx + t) : -1;
     }
-    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < kLoadBatch; ++u) {
+      if (b0 + 32 * u >= end) break;
+      const int t = b0 + 32 * u + lane;
+      const bool valid = t < end;
+      const int key = valid ? ((v[u] >= 0 && v[u] < S) ? v[u] : S) : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, key);
+      int pos = 0;
+      if (valid) pos = cnt[warp * K + key] + __popc(peers & lanemask_lt());
+      __syncwarp();
+      if (valid) {
+        perm[pos] = t;
+        if (lane == __ffs(peers) - 1) cnt[warp * K + key] += __popc(peers);
+      }
+      __syncwarp();
+    }
   }
 }
 
@@ -219,10 +308,25 @@ segment_items_kernel(int T, int S, int n_seg, const int32_t* __restrict__ seg_st
   }
 }
 
+// Per-slot ranks into the workspace (ranks == null clears them).
+__global__ void set_ranks_kernel(int S, const int32_t* __restrict__ ranks, char* __restrict__ meta) {
+  MetaHeader* hdr = reinterpret_cast<MetaHeader*>(meta);
+  int* dst = reinterpret_cast<int*>(meta + MetaLayout::a256(256) +
+                                    MetaLayout::a256(sizeof(int) * (size_t)(S + 2)));
+  if (ranks != nullptr)
+    for (int g = threadIdx.x; g < S; g += blockDim.x) dst[g] = ranks[g];
+  if (threadIdx.x == 0) hdr->has_ranks = ranks != nullptr ? 1 : 0;
+}
+
 }  // namespace
 
+cudaError_t launch_set_ranks(int S, const int32_t* ranks, void* meta, cudaStream_t st) {
+  set_ranks_kernel<<<1, 256, 0, st>>>(S, ranks, static_cast<char*>(meta));
+  return counted_launch(cudaGetLastError());
+}
+
 size_t group_smem_bytes(int S) {
-  return sizeof(int) * ((size_t)(kGroupWarps + 3) * (S + 1) + 65);
+  return sizeof(int) * ((size_t)(kGroupWarps + 4) * (S + 1) + 66);
 }
 
 cudaError_t launch_group(int T, int S, const int32_t* idx, void* meta, cudaStream_t st) {
@@ -230,7 +334,7 @@ cudaError_t launch_group(int T, int S, const int32_t* idx, void* meta, cudaStrea
   cudaError_t e = cudaFuncSetAttribute(group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  group_kernel<<<1, kGroupThreads, smem, st>>>(T, S, idx, static_cast<char*>(meta));
+  group_kernel<<<group_ctas(T), kGroupThreads, smem, st>>>(T, S, idx, static_cast<char*>(meta));
   return counted_launch(cudaGetLastError());
 }
 

@@ -76,6 +76,7 @@ bool bgmv_fused_fits(int T, int D, int r, int n_slices, const int32_t* D_out);
 cudaError_t launch_bgmv_fused(lora_dtype dt, const FusedArgs& a, cudaStream_t st);
 
 size_t group_smem_bytes(int S);
+cudaError_t launch_set_ranks(int S, const int32_t* ranks, void* meta, cudaStream_t st);
 cudaError_t launch_group(int T, int S, const int32_t* idx, void* meta, cudaStream_t st);
 cudaError_t launch_segment_items(int T, int S, int n_seg, const int32_t* seg_starts,
                                  const int32_t* seg_adapter, void* meta, cudaStream_t st);
@@ -95,6 +96,9 @@ cudaError_t launch_expand_segment_tc(lora_dtype dt, const ExpandArgs& a, const S
 // gathered through the token permutation).
 cudaError_t launch_shrink_grouped_tc(lora_dtype dt, const ShrinkArgs& a, cudaStream_t st);
 cudaError_t launch_expand_grouped_tc(lora_dtype dt, const ExpandArgs& a, cudaStream_t st);
+// Laned shrink: all slots' A as one [S*r, D] matrix on tensor cores, each
+// token's own lanes selected; needs no grouping.
+cudaError_t launch_shrink_laned(lora_dtype dt, const ShrinkArgs& a, cudaStream_t st);
 // Whether the per-token calls use the tensor-core kernels for this shape.
 inline bool grouped_tc_preferred(int T, int r, int S) { return r >= 16 && T >= 16 * S; }
 

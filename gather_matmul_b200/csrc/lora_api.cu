@@ -121,6 +121,16 @@ lora_status lora_group(int T, int S, const int32_t* idx, void* meta, size_t meta
   return from_cuda(launch_group(T, S, idx, meta, (cudaStream_t)stream));
 }
 
+lora_status lora_set_slot_ranks(int S, const int32_t* ranks, void* meta, size_t meta_bytes,
+                               lora_stream_t stream) {
+  if (S < 1 || S > LORA_MAX_SLOTS) return LORA_ERR_UNSUPPORTED;
+  if (meta == nullptr) return LORA_ERR_INVALID_ARG;
+  if (!aligned16(meta)) return LORA_ERR_MISALIGNED;
+  if (meta_bytes < lora_workspace_bytes(0, S)) return LORA_ERR_INVALID_ARG;
+  cudaGetLastError();
+  return from_cuda(launch_set_ranks(S, ranks, meta, (cudaStream_t)stream));
+}
+
 lora_status lora_shrink(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
                         const void* x, int64_t ldx, const void* const* A, const int32_t* idx,
                         float* buf, int has_active, const void* meta, size_t meta_bytes,
@@ -144,6 +154,31 @@ lora_status lora_shrink(lora_dtype dtype, int T, int D, int r, int S, int n_slic
     cudaGetLastError();
   }
   return from_cuda(launch_shrink_items(dtype, a, max_items_tokens(T, S), (cudaStream_t)stream));
+}
+
+lora_status lora_shrink_laned(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
+                              const void* x, int64_t ldx, const void* const* A,
+                              const int32_t* idx, float* buf, int has_active, void* meta,
+                              size_t meta_bytes, lora_stream_t stream) {
+  // only the workspace's error counters are used
+  if (meta == nullptr || meta_bytes < sizeof(MetaHeader)) return LORA_ERR_INVALID_ARG;
+  const size_t need = lora_workspace_bytes(T, S);
+  lora_status s = check_shrink(dtype, T, D, r, S, n_slices, x, ldx, A, buf, meta,
+                               need > meta_bytes ? need : meta_bytes);
+  if (s != LORA_OK) return s;
+  if (!has_active || T == 0) return LORA_OK;
+  if (idx == nullptr) return LORA_ERR_INVALID_ARG;
+  ShrinkArgs a = {};
+  a.x = x;
+  a.ldx = ldx;
+  for (int i = 0; i < n_slices; ++i) a.A[i] = A[i];
+  a.idx = idx;
+  a.buf = buf;
+  a.T = T; a.D = D; a.r = r; a.S = S; a.n_slices = n_slices;
+  a.meta = static_cast<const char*>(meta);
+  cudaGetLastError();
+  cudaError_t e = launch_shrink_laned(dtype, a, (cudaStream_t)stream);
+  return e == cudaErrorNotSupported ? LORA_ERR_UNSUPPORTED : from_cuda(e);
 }
 
 static void fill_expand(ExpandArgs& a, int T, int r, int S, int n_slices, const float* buf,
@@ -359,7 +394,7 @@ namespace {
 
 // Sized for LORA_NOALLOC_MAX_TOKENS tokens over LORA_MAX_SLOTS slots; every
 // GPU that loads the library holds it until the process exits.
-constexpr size_t kNoallocScratchBytes = 176896;
+constexpr size_t kNoallocScratchBytes = 197632;
 static_assert(kNoallocScratchBytes == LORA_NOALLOC_SCRATCH_BYTES, "header and library agree");
 static __device__ __align__(256) char g_noalloc_scratch[kNoallocScratchBytes];
 

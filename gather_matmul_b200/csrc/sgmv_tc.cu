@@ -136,6 +136,7 @@ struct ShrinkTCParams {
   CUtensorMap tmX;                       // x as [T rows, D cols], box {64, 128} (or {64, 1}
                                          // for row gathers), 128B swizzle
   CUtensorMap tmA[LORA_MAX_SLICES];      // A_i as [S*r rows, D cols], box {64, r}, 128B swizzle
+  CUtensorMap tmA8[LORA_MAX_SLICES];     // the same, box {64, 8}: a smaller slot rank, 8 rows a copy
   const int32_t* seg_starts;
   const int32_t* seg_adapter;
   int n_seg;
@@ -146,6 +147,7 @@ struct ShrinkTCParams {
   int T, D, S, n_slices, KS;
   int* bad_index;
   int* bad_meta;
+  const char* meta;                      // workspace: per-slot ranks
 };
 
 template <int R>
@@ -174,7 +176,6 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   using L = ShrinkSmem<R>;
   constexpr int kStages = L::kStages;
   constexpr bool kBF = std::is_same<E, __nv_bfloat16>::value;
-  constexpr uint32_t kIdesc = ptx::umma_idesc_f16(kBF, kTM, R);
   constexpr uint32_t kTmemCols = R < 32 ? 32 : R;
   cg::cluster_group cluster = cg::this_cluster();
   const int KS = P.KS;
@@ -233,6 +234,11 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   const int nkb_all = (P.D + kBK - 1) / kBK;
   const int kb0 = kr * nkb_all / KS, kb1 = (kr + 1) * nkb_all / KS;
   const int nkb = kb1 - kb0;                  // >= 1 (the host keeps KS <= nkb_all)
+  // the slot's own rank kk (a multiple of 8): only its first kk rows of A are
+  // read, and the MMA is N = kk rounded up to 16 wide
+  const int kk = slot_rank(P.meta, P.S, adapter, R);
+  const uint32_t idesc = ptx::umma_idesc_f16(kBF, kTM, kk < 16 ? 16 : (kk + 15) & ~15);
+  const uint32_t a_bytes = (uint32_t)kk * 128;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -279,10 +285,16 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
       const int mine = perm ? max((ngroups - warp + 3) / 4, 0) : 0;
       if (lane == 0) {
         uint32_t bytes = (uint32_t)(mine * 512);
-        if (warp == 0) bytes += (uint32_t)L::kABytes + (perm ? 0u : (uint32_t)L::kXBytes);
+        if (warp == 0) bytes += a_bytes + (perm ? 0u : (uint32_t)L::kXBytes);
         ptx::mbar_arrive_expect_tx(&full[s], bytes);
         if (warp == 0) {
-          ptx::tma_load_2d(st + L::kXBytes, &P.tmA[slice], kx, adapter * R, &full[s]);
+          if (kk == R) {
+            ptx::tma_load_2d(st + L::kXBytes, &P.tmA[slice], kx, adapter * R, &full[s]);
+          } else {
+            for (int b = 0; b < kk / 8; ++b)       // same layout as one kk-row box
+              ptx::tma_load_2d(st + L::kXBytes + b * 1024, &P.tmA8[slice], kx,
+                               adapter * R + 8 * b, &full[s]);
+          }
           if (!perm) ptx::tma_load_2d(st, &P.tmX, kx, m0, &full[s]);
         }
       }
@@ -302,7 +314,7 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
 #pragma unroll
       for (int k = 0; k < kBK / 16; ++k)
         ptx::tc_mma_f16(tmem, ptx::umma_desc_kmajor(xa + k * 32, 128),
-                        ptx::umma_desc_kmajor(aa + k * 32, 128), kIdesc, (i > 0 || k > 0) ? 1u : 0u);
+                        ptx::umma_desc_kmajor(aa + k * 32, 128), idesc, (i > 0 || k > 0) ? 1u : 0u);
       ptx::tc_commit(&empty[s]);              // stage s is free once these MMAs finish
     }
     ptx::tc_commit(accbar);
@@ -320,8 +332,9 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
       uint32_t r[16];
       ptx::tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c * 16, r);
       ptx::tc_wait_ld();
+      // columns past the slot's rank: zero (the accumulator holds nothing there)
 #pragma unroll
-      for (int u = 0; u < 16; ++u) v[c * 16 + u] = __uint_as_float(r[u]);
+      for (int u = 0; u < 16; ++u) v[c * 16 + u] = c * 16 + u < kk ? __uint_as_float(r[u]) : 0.f;
     }
   }
   if (KS == 1) {
@@ -379,6 +392,7 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
 //                quadrant split the columns (or the token chunks)
 struct ExpRun {
   int m0, valid, adapter, slice, j0, j1;
+  int kc;        // the adapter's rank rounded up to 16 << kc (per-slot ranks)
 };
 constexpr int kMaxRuns = 64;
 constexpr int kMaxSegTC = 2048;          // longer segment lists use the item kernels
@@ -387,7 +401,10 @@ constexpr int kSwapMax = 64;             // tiles of at most this many rows swap
 constexpr int kSegCache = 256;           // segment lists up to this long are read once
 
 struct ExpandTCParams {
-  CUtensorMap tmB[LORA_MAX_SLICES];      // B_i as [S*D_out_i rows, r cols], box {r, 128}
+  // B_i as [S*D_out_i rows, r cols], box {16 << c, 128} with a (32 << c)-byte
+  // swizzle: class c = 0, 1, 2 reads the first 16 / 32 / 64 columns of each
+  // row (a slot's own rank rounded up to 16; c <= log2(r / 16))
+  CUtensorMap tmB[3][LORA_MAX_SLICES];
   CUtensorMap tmY;                       // y as [T rows, ldy cols], box {64, 128}, 128B swizzle
   CUtensorMap tmYg;                      // y, box {64, 1}: 4-row gathers
   const float* buf;
@@ -406,6 +423,7 @@ struct ExpandTCParams {
   float scale;
   int* bad_index;
   int* bad_meta;
+  const char* meta;                      // workspace: per-slot ranks
 };
 
 template <int R>
@@ -512,10 +530,17 @@ __device__ __forceinline__ int64_t ceil_pos(int64_t num, int64_t w) {
 // Warp-cooperative: the tile runs whose pair start positions fall in
 // [lo, hi), in schedule order, at most kMaxRuns of them.  Returns the count;
 // *next is hi when the list is complete, else where the next list starts.
+// Rank class of an adapter: its rank rounded up to 16 << kc.
+template <int R>
+__device__ __forceinline__ int rank_class(const char* meta, int S, int adapter) {
+  const int k16 = max(16, (slot_rank(meta, S, adapter, R) + 15) & ~15);
+  return k16 == 16 ? 0 : (k16 == 32 ? 1 : 2);
+}
+
 template <int R>
 __device__ int build_runs(const SegView& sv, const int64_t* chunkW, int64_t Wt,
                           const int* ntiles, int n_slices, int64_t lo, int64_t hi,
-                          ExpRun* runs, int64_t* next) {
+                          ExpRun* runs, int64_t* next, const char* meta) {
   const int lane = threadIdx.x & 31;
   const int nch = (sv.n_seg + 31) / 32;
   int n = 0;
@@ -552,6 +577,7 @@ __device__ int build_runs(const SegView& sv, const int64_t* chunkW, int64_t Wt,
         const int len = __shfl_sync(0xffffffffu, b, l) - a_l;
         const int ad_l = __shfl_sync(0xffffffffu, ad, l);
         const int64_t sp = __shfl_sync(0xffffffffu, spos, l);
+        const int kc_l = rank_class<R>(meta, sv.S, ad_l);
         const int ntk = (len + kTM - 1) / kTM;
         for (int k0 = 0; k0 < ntk; k0 += 32) {
           const int k = k0 + lane;
@@ -564,7 +590,7 @@ __device__ int build_runs(const SegView& sv, const int64_t* chunkW, int64_t Wt,
           const unsigned hm = __ballot_sync(0xffffffffu, has);
           const int rank = __popc(hm & ((1u << lane) - 1));
           if (has && n + rank < kMaxRuns)
-            runs[n + rank] = ExpRun{a_l + k * kTM, valid, ad_l, i, jl, jh};
+            runs[n + rank] = ExpRun{a_l + k * kTM, valid, ad_l, i, jl, jh, kc_l};
           const int cnt = __popc(hm);
           if (n + cnt > kMaxRuns) {
             // the first run that did not fit starts the next list
@@ -673,7 +699,7 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   while (lo < hi) {
     if (warp == kExpMma) {
       int64_t nx;
-      const int n = build_runs<R>(sv, chunkW, Wt, ntiles, P.n_slices, lo, hi, runs, &nx);
+      const int n = build_runs<R>(sv, chunkW, Wt, ntiles, P.n_slices, lo, hi, runs, &nx, P.meta);
       if (lane == 0) {
         *sNRuns = n;
         sRange[3] = nx;
@@ -720,13 +746,15 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
           if (pq >= kYS) ok &= ptx::mbar_wait_ff(&empty[s], ((pq / kYS) - 1) & 1, sAbort);
           const int n0 = j * kNT;
           char* ys = sY + (size_t)s * L::kYBytes;
+          // the B tile holds only the first 16 << kc columns of each row
+          const uint32_t bbytes = (uint32_t)(kNT * (16 << rn.kc) * 2);
           const uint32_t bytes =
               (uint32_t)(my_ops * 512) +
-              (pw == 0 ? (uint32_t)L::kBBytes + (tiled ? (uint32_t)L::kYBytes : 0u) : 0u);
+              (pw == 0 ? bbytes + (tiled ? (uint32_t)L::kYBytes : 0u) : 0u);
           if (lane == 0) {
             ptx::mbar_arrive_expect_tx(&full[s], bytes);
             if (pw == 0) {
-              ptx::tma_load_2d(sB + (size_t)s * L::kBBytes, &P.tmB[rn.slice], 0,
+              ptx::tma_load_2d(sB + (size_t)s * L::kBBytes, &P.tmB[rn.kc][rn.slice], 0,
                                rn.adapter * Dout + n0, &full[s]);
               if (tiled) {
                 ptx::tma_load_2d(ys, &P.tmY, (int)(ycol0 + n0), rn.m0, &full[s]);
@@ -761,7 +789,7 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
           float mx = 0.f;
 #pragma unroll
           for (int q = 0; q < R / 4; ++q) {
-            f[q] = tok >= 0 ? brow[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+            f[q] = (tok >= 0 && 4 * q < (16 << rn.kc)) ? brow[q] : make_float4(0.f, 0.f, 0.f, 0.f);
             mx = fmaxf(fmaxf(fmaxf(mx, fabsf(f[q].x)), fmaxf(fabsf(f[q].y), fabsf(f[q].z))),
                        fabsf(f[q].w));
           }
@@ -812,13 +840,15 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
             ptx::tc_fence_after();
             const uint32_t bb = ptx::smem_u32(sB + (size_t)s * L::kBBytes);
             const uint32_t acc = tmem + a * kNT;
+            const int bsw = 32 << rn.kc;            // B tile row bytes = its swizzle
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
               const uint32_t op = half ? loA : hiA;
 #pragma unroll
               for (int ks = 0; ks < R / 16; ++ks) {
+                if (ks >= (1 << rn.kc)) break;      // K steps past the slot's rank
                 const uint64_t dOp = ptx::umma_desc_kmajor(op + ks * 32, L::kRowBytes);
-                const uint64_t dB = ptx::umma_desc_kmajor(bb + ks * 32, L::kRowBytes);
+                const uint64_t dB = ptx::umma_desc_kmajor(bb + ks * 32, bsw);
                 ptx::tc_mma_f16(acc, swap ? dB : dOp, swap ? dOp : dB, idesc,
                                 (half | ks) ? 1u : 0u);
               }
@@ -1044,9 +1074,13 @@ cudaError_t shrink_tc_launch(const ShrinkArgs& a, const SegArgs& sg, lora_dtype 
   for (int i = 0; i < a.n_slices; ++i) {
     e = encode_tmap_2d(&P.tmA[i], dt, a.A[i], (uint64_t)a.D, (uint64_t)a.S * R,
                        (uint64_t)a.D * 2, kBK, R, 128);
+    if (e == cudaSuccess)
+      e = encode_tmap_2d(&P.tmA8[i], dt, a.A[i], (uint64_t)a.D, (uint64_t)a.S * R,
+                         (uint64_t)a.D * 2, kBK, 8, 128);
     if (e != cudaSuccess) return e;
   }
   const MetaHeader* hdr = reinterpret_cast<const MetaHeader*>(a.meta);
+  P.meta = a.meta;
   P.seg_starts = sg.seg_starts;
   P.seg_adapter = sg.seg_adapter;
   P.n_seg = sg.n_seg;
@@ -1116,9 +1150,12 @@ cudaError_t expand_tc_launch(const ExpandArgs& a, const SegArgs& sg, lora_dtype 
   memset(&P, 0, sizeof(P));
   long sum_nt = 0;
   for (int i = 0; i < a.n_slices; ++i) {
-    cudaError_t e = encode_tmap_2d(&P.tmB[i], dt, a.B[i], (uint64_t)R,
-                                   (uint64_t)a.S * a.D_out[i], (uint64_t)R * 2, R, kNT, R * 2);
-    if (e != cudaSuccess) return e;
+    for (int c = 0; (16 << c) <= R; ++c) {
+      cudaError_t e = encode_tmap_2d(&P.tmB[c][i], dt, a.B[i], (uint64_t)R,
+                                     (uint64_t)a.S * a.D_out[i], (uint64_t)R * 2, 16 << c, kNT,
+                                     32 << c);
+      if (e != cudaSuccess) return e;
+    }
     P.y_col_off[i] = a.y_col_off[i];
     P.D_out[i] = a.D_out[i];
     sum_nt += (a.D_out[i] + kNT - 1) / kNT;
@@ -1148,6 +1185,7 @@ cudaError_t expand_tc_launch(const ExpandArgs& a, const SegArgs& sg, lora_dtype 
   P.scale = a.scale;
   P.bad_index = const_cast<int*>(&hdr->bad_index);
   P.bad_meta = const_cast<int*>(&hdr->bad_meta);
+  P.meta = a.meta;
   // one CTA per SM, never more CTAs than (tile, n-tile) pairs
   const long max_tiles = (a.T + kTM - 1) / kTM + sg.n_seg;
   const long pairs = max_tiles * sum_nt;

@@ -96,6 +96,16 @@ def workspace(T: int, S: int, device="cuda") -> torch.Tensor:
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
+def set_slot_ranks(ranks: Optional[torch.Tensor], S: int, meta: torch.Tensor, stream=None):
+    """Record each slot's own rank (device int32 [S]; None clears) in the
+    workspace: the kernels then skip the zero padding of smaller-rank slots."""
+    if ranks is not None:
+        if ranks.dtype != torch.int32 or not ranks.is_contiguous() or ranks.numel() != S:
+            raise TypeError("ranks must be a contiguous int32 tensor of one rank per slot")
+    _check("lora_set_slot_ranks", _lib.load().lora_set_slot_ranks(
+        int(S), _ptr(ranks), _ptr(meta), meta.numel(), _stream(stream)))
+
+
 def group(idx: torch.Tensor, S: int, meta: torch.Tensor, stream=None):
     """Group-by-slot metadata of one batch's int32 adapter indices (-1 = none)."""
     _check_idx(idx, idx.numel())
@@ -120,6 +130,21 @@ def shrink(x: torch.Tensor, A: Sequence[torch.Tensor], idx: torch.Tensor, buf: t
     S, r, _ = A[0].shape
     _check_idx(idx, T)
     _check("lora_shrink", _lib.load().lora_shrink(
+        _dtype(x), T, D, r, S, len(A), _ptr(x), ldx, _ptrs(A), _ptr(idx), _ptr(buf),
+        _active(has_active, idx_host, S), _ptr(meta), meta.numel(), _stream(stream)))
+    return buf
+
+
+def shrink_laned(x: torch.Tensor, A: Sequence[torch.Tensor], idx: torch.Tensor,
+                 buf: torch.Tensor, meta: torch.Tensor, has_active: Optional[bool] = None,
+                 idx_host=None, stream=None) -> torch.Tensor:
+    """shrink() without a grouping: every slot's lanes in one dense tensor-core
+    contraction, each token keeping its own slot's r lanes.  meta only
+    collects the error counters (group() is not needed)."""
+    T, D, ldx = _xinfo(x)
+    S, r, _ = A[0].shape
+    _check_idx(idx, T)
+    _check("lora_shrink_laned", _lib.load().lora_shrink_laned(
         _dtype(x), T, D, r, S, len(A), _ptr(x), ldx, _ptrs(A), _ptr(idx), _ptr(buf),
         _active(has_active, idx_host, S), _ptr(meta), meta.numel(), _stream(stream)))
     return buf

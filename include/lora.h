@@ -92,6 +92,28 @@ LORA_API size_t lora_workspace_bytes(int T, int S);
 LORA_API lora_status lora_workspace_reset(void* meta, size_t meta_bytes, lora_stream_t stream);
 
 /*
+ * Per-slot ranks ("Add multi-LoRA support", Features list: LoRAs of different
+ * ranks in one batch).  The stacks keep the call's rank r for every slot; a
+ * slot whose adapter has a smaller rank k fills only the first k rows of
+ * A_i[g] and the first k columns of B_i[g] and leaves the rest zero.  This
+ * records each slot's k in the workspace, so that the kernels skip the padded
+ * rows and columns (neither read nor multiplied) instead of multiplying
+ * zeros; the buf columns past a slot's rank are written as 0.
+ *
+ *   ranks   device int32 [S]: slot g's rank; 0, or a value >= the call's r,
+ *           means r.  Values are rounded up to a multiple of 8 (the padding
+ *           up to that multiple must be zero).  NULL clears the ranks.
+ *   meta    a workspace of at least lora_workspace_bytes(T, S) for the calls
+ *           that will use it; the ranks stay in it across lora_group calls
+ *           until changed, or until lora_workspace_reset.
+ * Enqueued on `stream` as one small kernel (capturable).  The fused one-launch
+ * path of lora_bgmv and lora_shrink_laned read the whole stack and ignore the
+ * ranks (the padding is zero, so their results are the same).
+ */
+LORA_API lora_status lora_set_slot_ranks(int S, const int32_t* ranks, void* meta,
+                                         size_t meta_bytes, lora_stream_t stream);
+
+/*
  * Group-by-slot metadata for one batch (the token-index tensor moved to the
  * device, as in pull 16989's review thread, then sorted by slot on the
  * device).  A stable counting sort of the tokens by idx[t]: tokens of slot 0
@@ -143,6 +165,32 @@ LORA_API lora_status lora_shrink(lora_dtype dtype, int T, int D, int r, int S, i
                         const void* x, int64_t ldx, const void* const* A, const int32_t* idx,
                         float* buf, int has_active, const void* meta, size_t meta_bytes,
                         lora_stream_t stream);
+
+/*
+ * Laned shrink: the same result as lora_group + lora_shrink, with no grouping
+ * and no sort.  After the LoRA laning of the TPU kernels in "[Hardware][TPU]
+ * [V1] Better tpu multilora compilation" (several adapters side by side in
+ * one register, one pass for tokens of different adapters): the stack A_i
+ * [S, r, D] is read as one [S*r, D] matrix of "lanes", every token is
+ * contracted with every lane on tcgen05 tensor cores (M = tokens, N = S*r,
+ * K = D, fp32 accumulator in tensor memory), and each token keeps the r lanes
+ * of its own slot: buf[i][t][j] = C[t][idx[t]*r + j].  The contraction does S
+ * times the useful multiply-adds; for small ranks and slot counts that stays
+ * far below the tensor-core roofline while x and A are read once, in dense
+ * tiles.
+ *
+ *   Arguments as for lora_shrink; idx is read directly (no lora_group);
+ *   indices outside [-1, S) are treated as -1 and counted.
+ *   meta   a workspace of at least 256 bytes whose error counters are used
+ *          (any lora_workspace_bytes-sized workspace will do).
+ * D must be a multiple of 8 and x 16-byte aligned with ldx a multiple of 8
+ * (tensor-map rules); otherwise LORA_ERR_MISALIGNED / LORA_ERR_UNSUPPORTED.
+ */
+LORA_API lora_status lora_shrink_laned(lora_dtype dtype, int T, int D, int r, int S,
+                                       int n_slices, const void* x, int64_t ldx,
+                                       const void* const* A, const int32_t* idx, float* buf,
+                                       int has_active, void* meta, size_t meta_bytes,
+                                       lora_stream_t stream);
 
 /*
  * BGMV expand into fused output slices (q/k/v, gate/up), one launch:
@@ -274,7 +322,7 @@ LORA_API lora_status lora_check_errors(void* meta, size_t meta_bytes, lora_strea
  *   the error counter).
  */
 #define LORA_NOALLOC_MAX_TOKENS 8192
-#define LORA_NOALLOC_SCRATCH_BYTES 176896
+#define LORA_NOALLOC_SCRATCH_BYTES 197632
 LORA_API lora_status lora_shrink_noalloc(lora_dtype dtype, int T, int D, int r, int S,
                                          int n_slices, const void* x, int64_t ldx,
                                          const void* const* A, const int32_t* idx, float* buf,
