@@ -27,6 +27,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -74,6 +75,8 @@ shrink_items_kernel(const ShrinkArgs a) {
   __shared__ float cpart[kItemTokens * kJR];
   __shared__ int stok[kItemTokens];
 
+  ptx::grid_dep_wait();               // the grouping / buf producers have finished
+  ptx::grid_dep_launch_dependents();
   cg::cluster_group cluster = cg::this_cluster();
   const int CL = (int)cluster.num_blocks();
   const int crank = (int)cluster.block_rank();
@@ -210,6 +213,8 @@ expand_items_kernel(const ExpandArgs a) {
   using YV = YVec<CPL>;
   constexpr int OC = kThreads * CPL;
 
+  ptx::grid_dep_wait();
+  ptx::grid_dep_launch_dependents();
   const int tid = threadIdx.x;
   MetaLayout L(a.T, a.S);
   const int n_items = checked_items(a.meta, a.T, a.S);
@@ -313,13 +318,14 @@ cudaError_t shrink_dispatch(const ShrinkArgs& a, int max_items, cudaStream_t st)
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CL;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return counted_launch(cudaLaunchKernelEx(&cfg, shrink_items_kernel<E>, a));
 }
 
@@ -328,8 +334,14 @@ cudaError_t expand_launch(const ExpandArgs& a, int max_items, cudaStream_t st) {
   long units = (long)max_items * a.chunk_base[a.n_slices];
   int grid = units < kPersistentCtas ? (int)units : kPersistentCtas;
   if (grid < 1) grid = 1;
-  expand_items_kernel<E, R, CPL><<<grid, kThreads, 0, st>>>(a);
-  return counted_launch(cudaGetLastError());
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return counted_launch(cudaLaunchKernelEx(&cfg, expand_items_kernel<E, R, CPL>, a));
 }
 
 template <typename E>

@@ -11,6 +11,7 @@
 // index_select copies).
 #include "common.cuh"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace lora {
 
@@ -109,6 +110,8 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
   int* ni = pre + K;                        // items per key, then item offsets
   int* scratch = ni + K;                    // 65 ints of scan scratch + a flag
 
+  ptx::grid_dep_wait();               // the previous kernel's writes (idx, meta) are visible
+  ptx::grid_dep_launch_dependents();
   MetaLayout L(T, S);
   MetaHeader* hdr = reinterpret_cast<MetaHeader*>(meta);
   int* slot_off = reinterpret_cast<int*>(meta + L.off_slot);
@@ -127,6 +130,9 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
   for (int i = tid; i < kGroupWarps * K; i += kGroupThreads) cnt[i] = 0;
   __syncthreads();
 
+  // a warp's first batch of indices stays in registers for the scatter pass
+  // (the only batch when the CTA has at most 32 * 32 * kLoadBatch tokens)
+  int v0[kLoadBatch];
   int bad = 0;
   for (int b0 = beg; b0 < end; b0 += 32 * kLoadBatch) {
     int v[kLoadBatch];
@@ -134,6 +140,10 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
     for (int u = 0; u < kLoadBatch; ++u) {
       const int t = b0 + 32 * u + lane;
       v[u] = t < end ? __ldg(idx + t) : -1;
+    }
+    if (b0 == beg) {
+#pragma unroll
+      for (int u = 0; u < kLoadBatch; ++u) v0[u] = v[u];
     }
 #pragma unroll
     for (int u = 0; u < kLoadBatch; ++u) {
@@ -220,7 +230,7 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
 #pragma unroll
     for (int u = 0; u < kLoadBatch; ++u) {
       const int t = b0 + 32 * u + lane;
-      v[u] = t < end ? __ldg(idx + t) : -1;
+      v[u] = b0 == beg ? v0[u] : (t < end ? __ldg(idx + t) : -1);
     }
 #pragma unroll
     for (int u = 0; u < kLoadBatch; ++u) {
@@ -250,6 +260,8 @@ segment_items_kernel(int T, int S, int n_seg, const int32_t* __restrict__ seg_st
   __shared__ int tile[2 * kGroupThreads];
   __shared__ int scratch[65];
   __shared__ int s_bad, s_carry;
+  ptx::grid_dep_wait();
+  ptx::grid_dep_launch_dependents();
   MetaLayout L(T, S);
   MetaHeader* hdr = reinterpret_cast<MetaHeader*>(meta);
   int4* items = reinterpret_cast<int4*>(meta + L.off_items);
@@ -334,15 +346,28 @@ cudaError_t launch_group(int T, int S, const int32_t* idx, void* meta, cudaStrea
   cudaError_t e = cudaFuncSetAttribute(group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  group_kernel<<<group_ctas(T), kGroupThreads, smem, st>>>(T, S, idx, static_cast<char*>(meta));
-  return counted_launch(cudaGetLastError());
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(group_ctas(T), 1, 1);
+  cfg.blockDim = dim3(kGroupThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return counted_launch(cudaLaunchKernelEx(&cfg, group_kernel, T, S, idx, static_cast<char*>(meta)));
 }
 
 cudaError_t launch_segment_items(int T, int S, int n_seg, const int32_t* seg_starts,
                                  const int32_t* seg_adapter, void* meta, cudaStream_t st) {
-  segment_items_kernel<<<1, kGroupThreads, 0, st>>>(T, S, n_seg, seg_starts, seg_adapter,
-                                                    static_cast<char*>(meta));
-  return counted_launch(cudaGetLastError());
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, 1, 1);
+  cfg.blockDim = dim3(kGroupThreads, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return counted_launch(cudaLaunchKernelEx(&cfg, segment_items_kernel, T, S, n_seg, seg_starts,
+                                           seg_adapter, static_cast<char*>(meta)));
 }
 
 }  // namespace lora

@@ -66,6 +66,17 @@ struct FusedArgs {
 // the library has made.
 cudaError_t counted_launch(cudaError_t e);
 
+// Launch attribute for programmatic dependent launch: the kernel may start
+// while the previous kernel on the stream runs; every kernel of the library
+// waits for its predecessor (griddepcontrol.wait) before it touches global
+// memory, then lets its own successor launch.
+inline cudaLaunchAttribute pdl_attribute() {
+  cudaLaunchAttribute a;
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+  return a;
+}
+
 cudaError_t encode_tmap_2d(CUtensorMap* map, lora_dtype dt, const void* base, uint64_t inner,
                            uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
                            uint32_t box_outer, int swizzle_bytes);

@@ -69,6 +69,8 @@ laned_shrink_kernel(const __grid_constant__ LanedParams P) {
   constexpr bool kBF = std::is_same<E, __nv_bfloat16>::value;
   constexpr uint32_t kIdesc = ptx::umma_idesc_f16(kBF, kLM, kLN);
   constexpr int kPitch = R + 4;                       // floats, received partial rows
+  ptx::grid_dep_wait();               // x, A and idx producers have finished
+  ptx::grid_dep_launch_dependents();
   cg::cluster_group cluster = cg::this_cluster();
   const int KS = P.KS;
   const int kr = (int)cluster.block_rank();
@@ -306,13 +308,14 @@ cudaError_t laned_launch(const ShrinkArgs& a, lora_dtype dt, cudaStream_t st) {
   cfg.blockDim = dim3(kLThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = KS;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return counted_launch(cudaLaunchKernelEx(&cfg, kern, P));
 }
 
