@@ -41,10 +41,9 @@ struct MetaHeader {
 };
 static_assert(sizeof(MetaHeader) == 256, "header is 256 bytes");
 
-// CTAs of the grouping kernel for T tokens: one per 8192 tokens (each of its
-// lanes then holds at most 8 indices in registers), at most 64 (all resident
-// at once, so they can meet at a barrier).
-constexpr int kGroupChunkMin = 8192;
+// CTAs of the grouping kernel for T tokens: one per 2048 tokens, at most 64
+// (all resident at once, so they can meet at a barrier).
+constexpr int kGroupChunkMin = 2048;
 constexpr int kGroupMaxCtas = 64;
 __host__ __device__ inline int group_ctas(int T) {
   const int nb = (T + kGroupChunkMin - 1) / kGroupChunkMin;

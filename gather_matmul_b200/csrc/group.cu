@@ -130,9 +130,6 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
   for (int i = tid; i < kGroupWarps * K; i += kGroupThreads) cnt[i] = 0;
   __syncthreads();
 
-  // a warp's first batch of indices stays in registers for the scatter pass
-  // (the only batch when the CTA has at most 32 * 32 * kLoadBatch tokens)
-  int v0[kLoadBatch];
   int bad = 0;
   for (int b0 = beg; b0 < end; b0 += 32 * kLoadBatch) {
     int v[kLoadBatch];
@@ -140,10 +137,6 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
     for (int u = 0; u < kLoadBatch; ++u) {
       const int t = b0 + 32 * u + lane;
       v[u] = t < end ? __ldg(idx + t) : -1;
-    }
-    if (b0 == beg) {
-#pragma unroll
-      for (int u = 0; u < kLoadBatch; ++u) v0[u] = v[u];
     }
 #pragma unroll
     for (int u = 0; u < kLoadBatch; ++u) {
@@ -230,7 +223,7 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
 #pragma unroll
     for (int u = 0; u < kLoadBatch; ++u) {
       const int t = b0 + 32 * u + lane;
-      v[u] = b0 == beg ? v0[u] : (t < end ? __ldg(idx + t) : -1);
+      v[u] = t < end ? __ldg(idx + t) : -1;
     }
 #pragma unroll
     for (int u = 0; u < kLoadBatch; ++u) {

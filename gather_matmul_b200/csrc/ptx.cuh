@@ -44,18 +44,6 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // other warps of the SM need.
 constexpr uint32_t kWaitSuspendNs = 1000000;
 
-// Whether the phase with the given parity has completed (no waiting).
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait for the phase with the given parity to complete.  Gives up after
 // about one second and returns false (the caller records an error and stops
 // instead of hanging the GPU).

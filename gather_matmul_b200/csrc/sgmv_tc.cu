@@ -377,6 +377,40 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   if (!ok && tid == 0) atomicAdd(P.bad_meta, 1);
 }
 
+constexpr int kMaxSegTC = 2048;          // longer segment lists use the item kernels
+constexpr int kMaxSegChunks = kMaxSegTC / 32 + 1;
+constexpr int kSegCache = 256;           // segment lists up to this long are read once
+
+struct SegView {
+  const int32_t* ss;
+  const int32_t* sa;
+  int n_seg, T, S, implicit_slots;
+  int4* cache;                           // shared-memory copy of the first kSegCache segments
+  // the same, from the copy when the whole list is in it
+  __device__ __forceinline__ void get_cached(int s, int& a, int& b, int& ad) const {
+    if (n_seg <= kSegCache) {
+      const int4 c = s < n_seg ? cache[s] : make_int4(0, 0, -1, 0);
+      a = c.x; b = c.y; ad = c.z;
+    } else {
+      get(s, a, b, ad);
+    }
+  }
+  // segment s clamped into [0, T]; adapter -1 when it has none or is out of range
+  __device__ __forceinline__ void get(int s, int& a, int& b, int& ad) const {
+    a = 0; b = 0; ad = -1;
+    if (s < n_seg) {
+      a = min(max(ss[s], 0), T);
+      b = max(a, min(max(ss[s + 1], 0), T));
+      ad = implicit_slots ? (s < implicit_slots ? s : -1) : sa[s];
+      if (ad < 0 || ad >= S) ad = -1;
+    }
+  }
+};
+
+__device__ __forceinline__ int64_t ceil_pos(int64_t num, int64_t w) {
+  return num <= 0 ? 0 : (num + w - 1) / w;
+}
+
 // ---------------------------------------------------------------- expand
 // Persistent: one CTA per SM walks a contiguous range of (slice, tile, n-tile)
 // pairs.  The pairs are ordered slice-major, then by tile, then by 128-column
@@ -396,20 +430,9 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
 struct ExpRun {
   int m0, valid, adapter, slice, j0, j1;
   int kc;        // the adapter's rank rounded up to 16 << kc (per-slot ranks)
-  int wide;      // output n-tiles per pair: 2 for tiles of <= kWideMax rows, else 1
 };
 constexpr int kMaxRuns = 64;
-constexpr int kMaxSegTC = 2048;          // longer segment lists use the item kernels
-constexpr int kMaxSegChunks = kMaxSegTC / 32 + 1;
 constexpr int kSwapMax = 64;             // tiles of at most this many rows swap operands
-// Tiles of at most kWideMax rows take 256 output columns per pair: two MMAs
-// into one accumulator, y as four 64-column blocks of <= 32 rows in the first
-// half of the stage's y region and the second B tile in its second half, so
-// that a pipeline stage of a small slot group moves twice the bytes.
-constexpr int kWideMax = 32;
-constexpr int kWideQ = kWideMax * 128;   // bytes of one 64-column y block of a wide pair
-constexpr int kWideBOff = 4 * kWideQ;    // the second B tile within the y region
-constexpr int kSegCache = 256;           // segment lists up to this long are read once
 
 struct ExpandTCParams {
   // B_i as [S*D_out_i rows, r cols], box {16 << c, 128} with a (32 << c)-byte
@@ -469,39 +492,6 @@ template <int R>
 __device__ __forceinline__ int64_t pair_weight(int valid) {
   return (int64_t)kNT * R * 2 + 512 * (int64_t)valid + 16384;
 }
-// The same per 128-column n-tile: a wide pair spreads its fixed cost over
-// its two n-tiles.
-template <int R>
-__device__ __forceinline__ int64_t ntile_weight(int valid) {
-  return valid <= kWideMax ? (int64_t)kNT * R * 2 + 512 * (int64_t)valid + 8192
-                           : pair_weight<R>(valid);
-}
-
-struct SegView {
-  const int32_t* ss;
-  const int32_t* sa;
-  int n_seg, T, S, implicit_slots;
-  int4* cache;                           // shared-memory copy of the first kSegCache segments
-  // the same, from the copy when the whole list is in it
-  __device__ __forceinline__ void get_cached(int s, int& a, int& b, int& ad) const {
-    if (n_seg <= kSegCache) {
-      const int4 c = s < n_seg ? cache[s] : make_int4(0, 0, -1, 0);
-      a = c.x; b = c.y; ad = c.z;
-    } else {
-      get(s, a, b, ad);
-    }
-  }
-  // segment s clamped into [0, T]; adapter -1 when it has none or is out of range
-  __device__ __forceinline__ void get(int s, int& a, int& b, int& ad) const {
-    a = 0; b = 0; ad = -1;
-    if (s < n_seg) {
-      a = min(max(ss[s], 0), T);
-      b = max(a, min(max(ss[s + 1], 0), T));
-      ad = implicit_slots ? (s < implicit_slots ? s : -1) : sa[s];
-      if (ad < 0 || ad >= S) ad = -1;
-    }
-  }
-};
 
 // Per n-tile weight of one segment: its full tiles and its partial last tile.
 template <int R>
@@ -509,21 +499,13 @@ __device__ __forceinline__ int64_t seg_weight(int a, int b, int ad) {
   if (ad < 0) return 0;
   const int len = b - a;
   const int rem = len % kTM;
-  return (int64_t)(len / kTM) * ntile_weight<R>(kTM) + (rem ? ntile_weight<R>(rem) : 0);
+  return (int64_t)(len / kTM) * pair_weight<R>(kTM) + (rem ? pair_weight<R>(rem) : 0);
 }
 
-// Rank class of an adapter: its rank rounded up to 16 << kc.
+// Warp 0 of the CTA: per-chunk (32 segments) weights into chunkW, total
+// returned in every lane.
 template <int R>
-__device__ __forceinline__ int rank_class(const char* meta, int S, int adapter) {
-  const int k16 = max(16, (slot_rank(meta, S, adapter, R) + 15) & ~15);
-  return k16 == 16 ? 0 : (k16 == 32 ? 1 : 2);
-}
-
-// One warp of the CTA: per-chunk (32 segments) weights into chunkW, total
-// returned in every lane; the first kSegCache segments, with their adapters'
-// rank classes, copied into shared memory.
-template <int R>
-__device__ int64_t seg_chunk_weights(const SegView& sv, int64_t* chunkW, const char* meta) {
+__device__ int64_t seg_chunk_weights(const SegView& sv, int64_t* chunkW) {
   const int lane = threadIdx.x & 31;
   const int nch = (sv.n_seg + 31) / 32;
   int64_t total = 0;
@@ -534,8 +516,7 @@ __device__ int64_t seg_chunk_weights(const SegView& sv, int64_t* chunkW, const c
       int a, b, ad;
       const int sidx = (c0 + u) * 32 + lane;
       sv.get(sidx, a, b, ad);
-      if (sidx < kSegCache)
-        sv.cache[sidx] = make_int4(a, b, ad, ad >= 0 ? rank_class<R>(meta, sv.S, ad) : 0);
+      if (sidx < kSegCache) sv.cache[sidx] = make_int4(a, b, ad, 0);
       w[u] = seg_weight<R>(a, b, ad);
     }
 #pragma unroll
@@ -550,13 +531,16 @@ __device__ int64_t seg_chunk_weights(const SegView& sv, int64_t* chunkW, const c
   return total;
 }
 
-__device__ __forceinline__ int64_t ceil_pos(int64_t num, int64_t w) {
-  return num <= 0 ? 0 : (num + w - 1) / w;
-}
 
 // Warp-cooperative: the tile runs whose pair start positions fall in
 // [lo, hi), in schedule order, at most kMaxRuns of them.  Returns the count;
 // *next is hi when the list is complete, else where the next list starts.
+// Rank class of an adapter: its rank rounded up to 16 << kc.
+template <int R>
+__device__ __forceinline__ int rank_class(const char* meta, int S, int adapter) {
+  const int k16 = max(16, (slot_rank(meta, S, adapter, R) + 15) & ~15);
+  return k16 == 16 ? 0 : (k16 == 32 ? 1 : 2);
+}
 
 template <int R>
 __device__ int build_runs(const SegView& sv, const int64_t* chunkW, int64_t Wt,
@@ -598,26 +582,20 @@ __device__ int build_runs(const SegView& sv, const int64_t* chunkW, int64_t Wt,
         const int len = __shfl_sync(0xffffffffu, b, l) - a_l;
         const int ad_l = __shfl_sync(0xffffffffu, ad, l);
         const int64_t sp = __shfl_sync(0xffffffffu, spos, l);
-        const int kc_l = c * 32 + l < kSegCache && sv.n_seg <= kSegCache
-                             ? sv.cache[c * 32 + l].w
-                             : rank_class<R>(meta, sv.S, ad_l);
+        const int kc_l = rank_class<R>(meta, sv.S, ad_l);
         const int ntk = (len + kTM - 1) / kTM;
         for (int k0 = 0; k0 < ntk; k0 += 32) {
           const int k = k0 + lane;
           const int valid = k < ntk ? min(kTM, len - k * kTM) : 0;
-          // pairs of this tile: wf n-tiles each, the pair's position is its
-          // first n-tile's
-          const int wf = valid <= kWideMax ? 2 : 1;
-          const int64_t npairs = (nt + wf - 1) / wf;
-          const int64_t step = wf * ntile_weight<R>(valid);
-          const int64_t tpos = sp + nt * (int64_t)k * ntile_weight<R>(kTM);
-          const int jl = (int)(ceil_pos(lo - tpos, step) < npairs ? ceil_pos(lo - tpos, step) : npairs);
-          const int jh = (int)(ceil_pos(hi - tpos, step) < npairs ? ceil_pos(hi - tpos, step) : npairs);
+          const int64_t w = pair_weight<R>(valid);
+          const int64_t tpos = sp + nt * (int64_t)k * pair_weight<R>(kTM);
+          const int jl = (int)(ceil_pos(lo - tpos, w) < nt ? ceil_pos(lo - tpos, w) : nt);
+          const int jh = (int)(ceil_pos(hi - tpos, w) < nt ? ceil_pos(hi - tpos, w) : nt);
           const bool has = k < ntk && jl < jh;
           const unsigned hm = __ballot_sync(0xffffffffu, has);
           const int rank = __popc(hm & ((1u << lane) - 1));
           if (has && n + rank < kMaxRuns)
-            runs[n + rank] = ExpRun{a_l + k * kTM, valid, ad_l, i, jl, jh, kc_l, wf};
+            runs[n + rank] = ExpRun{a_l + k * kTM, valid, ad_l, i, jl, jh, kc_l};
           const int cnt = __popc(hm);
           if (n + cnt > kMaxRuns) {
             // the first run that did not fit starts the next list
@@ -688,7 +666,7 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
     ptx::tmem_relinquish();
     // this CTA's share of the weighted pair sequence (the segment reads stay in
     // bounds whatever the workspace holds, so they need not wait for the check)
-    const int64_t Wt0 = seg_chunk_weights<R>(sv, chunkW, P.meta);
+    const int64_t Wt0 = seg_chunk_weights<R>(sv, chunkW);
     const bool meta_ok = !P.implicit_slots || grouped_meta_ok(P.bad_index, P.T, P.S, lane == 0);
     const int64_t Wt = meta_ok ? Wt0 : 0;
     const int64_t W = Wt * sum_nt;
@@ -742,30 +720,21 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
       // ---------------- loads
       const int pw = warp - kExpLoad0;
       const int lt = pw * 32 + lane;                 // operand row of this thread
-      const int m = lt;
       int pl = p, ul = u;
-      // this thread's row of a run: its token and (per-token grouping) the
-      // token's index; the next run's are fetched while this one is issued
-      auto fetch_row = [&](const ExpRun& r, int& tk, int& iv) {
-        tk = m < r.valid ? (P.perm ? P.perm[r.m0 + m] : r.m0 + m) : -1;
-        iv = (tk >= 0 && P.perm) ? P.idx[tk] : 0;
-      };
-      int tok_next = -1, idx_next = 0;
-      if (n_runs > 0) fetch_row(runs[0], tok_next, idx_next);
       for (int ri = 0; ri < n_runs; ++ri, ++ul) {
         const ExpRun rn = runs[ri];
         const int hb = ul & 1;
-        int tok = tok_next;
-        const int tok_idx = idx_next;
-        if (ri + 1 < n_runs) fetch_row(runs[ri + 1], tok_next, idx_next);
         if (ul >= 2) ok &= ptx::mbar_wait_ff(&hlempty[hb], ((ul >> 1) - 1) & 1, sAbort);
-        // the tokens first (the gathers need every row's token), then the
-        // loads of the run's pairs whose stages are already free, then the
-        // hi / lo rows, so that the buf reads overlap those loads.
+        // this thread's operand row: its token first (the gathers need every
+        // row's token), then the loads of the run's first pairs whose stages
+        // are free without waiting, then the hi / lo rows, so that the buf
+        // reads overlap those loads
+        const int m = lt;
         // sTok: the row's token; -1 past the tile; -2 - token for a token whose
         // index disagrees with its group (stale workspace): still a valid row
         // address for the gathers, but never written back (counted here)
-        if (tok >= 0 && P.perm && tok_idx != rn.adapter) {
+        int tok = m < rn.valid ? (P.perm ? P.perm[rn.m0 + m] : rn.m0 + m) : -1;
+        if (tok >= 0 && P.perm && !grouped_row_ok(P.idx, tok, rn.adapter, P.S)) {
           if (rn.j0 == 0) atomicAdd(P.bad_meta, 1);
           tok = -2 - tok;
         }
@@ -776,27 +745,24 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
         const int64_t ycol0 = P.y_col_off[rn.slice];
         const bool tiled = P.perm == nullptr && rn.valid == kTM;
         const int ngroups = (rn.valid + 3) / 4;
-        const bool wide = rn.wide == 2;
-        const int nops = (wide ? 4 : 2) * ngroups;   // 4-row gathers: 64-column blocks x groups
-        const int my_ops = tiled ? 0 : max((nops - pw + 3) / 4, 0);
+        int my_ops = 0;
+        if (!tiled)
+          for (int o = pw; o < 2 * ngroups; o += 4) ++my_ops;
         auto issue_pair = [&](int j, int pq) {
           const int s = pq % kYS;
           if (pq >= kYS) ok &= ptx::mbar_wait_ff(&empty[s], ((pq / kYS) - 1) & 1, sAbort);
-          const int n0 = j * rn.wide * kNT;
+          const int n0 = j * kNT;
           char* ys = sY + (size_t)s * L::kYBytes;
           // the B tile holds only the first 16 << kc columns of each row
           const uint32_t bbytes = (uint32_t)(kNT * (16 << rn.kc) * 2);
           const uint32_t bytes =
               (uint32_t)(my_ops * 512) +
-              (pw == 0 ? rn.wide * bbytes + (tiled ? (uint32_t)L::kYBytes : 0u) : 0u);
+              (pw == 0 ? bbytes + (tiled ? (uint32_t)L::kYBytes : 0u) : 0u);
           if (lane == 0) {
             ptx::mbar_arrive_expect_tx(&full[s], bytes);
             if (pw == 0) {
               ptx::tma_load_2d(sB + (size_t)s * L::kBBytes, &P.tmB[rn.kc][rn.slice], 0,
                                rn.adapter * Dout + n0, &full[s]);
-              if (wide)       // rows past this slot's D_out feed columns never stored
-                ptx::tma_load_2d(ys + kWideBOff, &P.tmB[rn.kc][rn.slice], 0,
-                                 rn.adapter * Dout + n0 + kNT, &full[s]);
               if (tiled) {
                 ptx::tma_load_2d(ys, &P.tmY, (int)(ycol0 + n0), rn.m0, &full[s]);
                 ptx::tma_load_2d(ys + L::kYHalf, &P.tmY, (int)(ycol0 + n0 + 64), rn.m0, &full[s]);
@@ -805,29 +771,22 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
           }
           __syncwarp();
           if (!tiled) {
-            // 64-column blocks x ngroups 4-row gathers: op o -> warp o % 4,
-            // lane o / 4; a wide pair's block b holds <= 32 rows at b * kWideQ
-            for (int o = pw + 4 * lane; o < nops; o += 128) {
-              const int g = wide ? o >> 2 : o >> 1, h = wide ? o & 3 : o & 1;
+            // 2 halves x ngroups 4-row gathers: op o -> warp o % 4, lane o / 4
+            for (int o = pw + 4 * lane; o < 2 * ngroups; o += 128) {
+              const int g = o >> 1, h = o & 1;
               int rr[4];
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const int t = toks[4 * g + q < rn.valid ? 4 * g + q : 4 * g];
                 rr[q] = t >= 0 ? t : -2 - t;
               }
-              ptx::tma_gather4(ys + h * (wide ? kWideQ : L::kYHalf) + g * 512, &P.tmYg,
-                               (int)(ycol0 + n0 + 64 * h), rr[0], rr[1], rr[2], rr[3], &full[s]);
+              ptx::tma_gather4(ys + h * L::kYHalf + g * 512, &P.tmYg, (int)(ycol0 + n0 + 64 * h),
+                               rr[0], rr[1], rr[2], rr[3], &full[s]);
             }
           }
         };
-        // every pair whose stage is free now; the four load warps may decide
-        // differently, which is harmless: each warp still arrives once per
-        // pair, in pair order, and issues only its own copies
         int j = rn.j0;
-        for (; j < rn.j1; ++j, ++pl) {
-          if (pl >= kYS && !ptx::mbar_test(&empty[pl % kYS], ((pl / kYS) - 1) & 1)) break;
-          issue_pair(j, pl);
-        }
+        for (; j < rn.j1 && pl < kYS; ++j, ++pl) issue_pair(j, pl);
         // hi / lo after an exact power-of-two rescale 2^(7-e) (e = exponent of
         // the row's max |buf|), and the inverse scale
         {
@@ -886,24 +845,19 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
             ok &= ptx::mbar_wait_ff(&full[s], (pl / kYS) & 1, sAbort);
             if (pl >= 2) ok &= ptx::mbar_wait_ff(&accempty[a], ((pl >> 1) - 1) & 1, sAbort);
             ptx::tc_fence_after();
+            const uint32_t bb = ptx::smem_u32(sB + (size_t)s * L::kBBytes);
+            const uint32_t acc = tmem + a * kNT;
             const int bsw = 32 << rn.kc;            // B tile row bytes = its swizzle
-            // a wide pair: the second 128 columns from the B tile in the y
-            // region, into accumulator columns 64.. (N <= 32)
-            for (int c = 0; c < rn.wide; ++c) {
-              const uint32_t bb = c == 0 ? ptx::smem_u32(sB + (size_t)s * L::kBBytes)
-                                         : ptx::smem_u32(sY + (size_t)s * L::kYBytes + kWideBOff);
-              const uint32_t acc = tmem + a * kNT + c * 64;
 #pragma unroll
-              for (int half = 0; half < 2; ++half) {
-                const uint32_t op = half ? loA : hiA;
+            for (int half = 0; half < 2; ++half) {
+              const uint32_t op = half ? loA : hiA;
 #pragma unroll
-                for (int ks = 0; ks < R / 16; ++ks) {
-                  if (ks >= (1 << rn.kc)) break;    // K steps past the slot's rank
-                  const uint64_t dOp = ptx::umma_desc_kmajor(op + ks * 32, L::kRowBytes);
-                  const uint64_t dB = ptx::umma_desc_kmajor(bb + ks * 32, bsw);
-                  ptx::tc_mma_f16(acc, swap ? dB : dOp, swap ? dOp : dB, idesc,
-                                  (half | ks) ? 1u : 0u);
-                }
+              for (int ks = 0; ks < R / 16; ++ks) {
+                if (ks >= (1 << rn.kc)) break;      // K steps past the slot's rank
+                const uint64_t dOp = ptx::umma_desc_kmajor(op + ks * 32, L::kRowBytes);
+                const uint64_t dB = ptx::umma_desc_kmajor(bb + ks * 32, bsw);
+                ptx::tc_mma_f16(acc, swap ? dB : dOp, swap ? dOp : dB, idesc,
+                                (half | ks) ? 1u : 0u);
               }
             }
             ptx::tc_commit(&accfull[a]);
@@ -935,7 +889,7 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
           // lane quadrant), the group of its accumulator: consecutive small
           // pairs overlap; a full pair by all eight
           if (swap && a != h) continue;
-          const int n0 = j * rn.wide * kNT, nn = min(rn.wide * kNT, Dout - n0);
+          const int n0 = j * kNT, nn = min(kNT, Dout - n0);
           ok &= ptx::mbar_wait_ff(&accfull[a], (pl >> 1) & 1, sAbort);
           ok &= ptx::mbar_wait_ff(&full[s], (pl / kYS) & 1, sAbort);
           ptx::tc_fence_after();
@@ -1019,18 +973,14 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
               ptx::fence_proxy_async_smem();
             }
           } else {
-            // swapped: thread = output column 32q + lane of each 128-column
-            // MMA tile c, all groups of 8 tokens; y in 64-column blocks
-            // kYHalf apart (a wide pair's <= 32 rows: kWideQ apart)
-            const bool wide = rn.wide == 2;
+            // swapped: thread = output column 32q + lane, all groups of 8 tokens
+            const int col = q * 32 + lane;
+            const int hc = col >> 6, cc = col & 63;
+            char* cbase = ys + hc * L::kYHalf + (cc & 7) * 2;
             const int ng = (rn.valid + 7) / 8;
-            for (int cg = 0; cg < rn.wide * ng; ++cg) {
-              const int c = cg / ng, g = cg % ng;
-              const int col = c * kNT + q * 32 + lane;
-              const int hc = col >> 6, cc = col & 63;
-              char* cbase = ys + hc * (wide ? kWideQ : L::kYHalf) + (cc & 7) * 2;
+            for (int g = 0; g < ng; ++g) {
               uint32_t r[8];
-              ptx::tc_ld8(tacc + c * 64 + 8 * g, r);
+              ptx::tc_ld8(tacc + 8 * g, r);
               const float4 i0 = *reinterpret_cast<const float4*>(invs + 8 * g);
               const float4 i1 = *reinterpret_cast<const float4*>(invs + 8 * g + 4);
               const float iv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
@@ -1054,25 +1004,21 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive_cnt(&accempty[a], 2);   // four warps count as eight
             asm volatile("bar.sync %0, 128;" ::"r"(1 + h) : "memory");   // the group's columns done
-            // rows 0 .. valid-1, 16 chunks each (wide: 32): e -> (row, 64-column
-            // block, chunk); at most 64 (wide: 32) rows: eight pieces per
-            // thread, all read before any store
+            // rows 0 .. valid-1, 16 chunks each: e -> (row e / 16, chunk e % 16);
+            // at most 64 rows: eight pieces per thread, all read before any store
             const int gl = q * 32 + lane;
-            const int cshift = wide ? 5 : 4, bmask = wide ? 3 : 1;
-            const int bstride = wide ? kWideQ : L::kYHalf;
-            const int rmax = wide ? kWideMax - 1 : kSwapMax - 1;
             uint4 v[8];
 #pragma unroll
             for (int it = 0; it < 8; ++it) {
               const int e = gl + 128 * it;
-              const int mr = min(e >> cshift, rmax), hh = (e >> 3) & bmask, ch = e & 7;
-              v[it] = *reinterpret_cast<const uint4*>(ys + hh * bstride + mr * 128 +
+              const int mr = min(e >> 4, kSwapMax - 1), hh = (e >> 3) & 1, ch = e & 7;
+              v[it] = *reinterpret_cast<const uint4*>(ys + hh * L::kYHalf + mr * 128 +
                                                       ((ch ^ (mr & 7)) << 4));
             }
 #pragma unroll
             for (int it = 0; it < 8; ++it) {
               const int e = gl + 128 * it;
-              const int mr = e >> cshift, hh = (e >> 3) & bmask, ch = e & 7;
+              const int mr = e >> 4, hh = (e >> 3) & 1, ch = e & 7;
               if (mr < rn.valid && 64 * hh + 8 * ch < nn && toks[mr] >= 0)
                 *reinterpret_cast<uint4*>(ycol + (size_t)toks[mr] * P.ldy + n0 + 64 * hh + 8 * ch) =
                     v[it];

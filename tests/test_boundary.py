@@ -210,12 +210,12 @@ def test_integer_inputs_match_oracle_bitwise(dt, D, r):
                                       (W.BF16, 8, 200, 3), (W.BF16, 8, 300, 2),
                                       (W.F16, 64, 200, 8), (W.BF16, 8, 260, 12)],
                          ids=["f16-small-groups", "f16-full-tiles", "bf16-small-groups",
-                              "bf16-full-tiles", "f16-wide-pairs", "bf16-wide-pairs"])
+                              "bf16-full-tiles", "f16-many-slots", "bf16-many-slots"])
 def test_integer_inputs_grouped_tensor_cores_bitwise(dt, D, T, S):
     # T >= 16 S with r = 16: the per-token batch runs through the grouping on
     # the tcgen05 kernels (groups of about 50 rows take the operand-swapped
-    # expand, about 100 rows the full 128-row tile, about 20 rows the wide
-    # 256-column pairs).  x, A, B in {-1,0,1},
+    # expand, about 100 rows the full 128-row tile, about 20 rows the
+    # swapped tile with few rows).  x, A, B in {-1,0,1},
     # y in [-8,8]: |buf| <= D and |y| <= 8 + 16 D stay exact (fp16: <= 1032
     # < 2048; bf16: <= 136 < 256), through the hi + lo split as well, so the
     # GPU equals the oracle bit for bit.
