@@ -33,6 +33,11 @@ struct ExpandArgs {
   int64_t ldy;
   int T, r, S, n_slices;
   const char* meta;
+  // 1: the kernel launched just before on the stream is this library's shrink
+  // of the same batch (it writes only buf and the error counters), so the
+  // tensor-core expand may read the grouping, B and y before that kernel has
+  // finished and waits for it only before reading buf
+  int after_shrink;
 };
 
 struct SegArgs {

@@ -200,11 +200,14 @@ static void fill_expand(ExpandArgs& a, int T, int r, int S, int n_slices, const 
   a.meta = static_cast<const char*>(meta);
 }
 
-lora_status lora_expand(lora_dtype dtype, int T, int r, int S, int n_slices,
-                        const float* buf, int64_t buf_slice_stride, const void* const* B,
-                        const int32_t* D_out, const int32_t* idx, float scale, void* y,
-                        int64_t ldy, const int64_t* y_col_off, int has_active, const void* meta,
-                        size_t meta_bytes, lora_stream_t stream) {
+// after_shrink: the previous launch on the stream is lora_shrink's kernel for
+// this batch (lora_bgmv's three-launch path)
+static lora_status expand_impl(lora_dtype dtype, int T, int r, int S, int n_slices,
+                               const float* buf, int64_t buf_slice_stride, const void* const* B,
+                               const int32_t* D_out, const int32_t* idx, float scale, void* y,
+                               int64_t ldy, const int64_t* y_col_off, int has_active,
+                               const void* meta, size_t meta_bytes, lora_stream_t stream,
+                               int after_shrink) {
   lora_status s = check_expand(dtype, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, y,
                                ldy, y_col_off, meta, meta_bytes);
   if (s != LORA_OK) return s;
@@ -213,6 +216,7 @@ lora_status lora_expand(lora_dtype dtype, int T, int r, int S, int n_slices,
   ExpandArgs a = {};
   fill_expand(a, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, idx, scale, y, ldy,
               y_col_off, meta);
+  a.after_shrink = after_shrink;
   cudaGetLastError();
   if (grouped_tc_preferred(T, r, S)) {
     cudaError_t e = launch_expand_grouped_tc(dtype, a, (cudaStream_t)stream);
@@ -220,6 +224,15 @@ lora_status lora_expand(lora_dtype dtype, int T, int r, int S, int n_slices,
     cudaGetLastError();
   }
   return from_cuda(launch_expand_items(dtype, a, max_items_tokens(T, S), (cudaStream_t)stream));
+}
+
+lora_status lora_expand(lora_dtype dtype, int T, int r, int S, int n_slices,
+                        const float* buf, int64_t buf_slice_stride, const void* const* B,
+                        const int32_t* D_out, const int32_t* idx, float scale, void* y,
+                        int64_t ldy, const int64_t* y_col_off, int has_active, const void* meta,
+                        size_t meta_bytes, lora_stream_t stream) {
+  return expand_impl(dtype, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, idx, scale, y,
+                     ldy, y_col_off, has_active, meta, meta_bytes, stream, 0);
 }
 
 lora_status lora_shrink_segment(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
@@ -330,10 +343,12 @@ lora_status lora_bgmv(lora_dtype dtype, int T, int D, int r, int S, int n_slices
   cudaGetLastError();
   s = lora_group(T, S, idx, meta, meta_bytes, stream);
   if (s != LORA_OK) return s;
+  // a successful lora_shrink is exactly one launch on `stream`: the expand's
+  // predecessor
   s = lora_shrink(dtype, T, D, r, S, n_a, x, ldx, A, idx, buf, 1, meta, meta_bytes, stream);
   if (s != LORA_OK) return s;
-  return lora_expand(dtype, T, r, S, n_slices, buf, shared_A ? 0 : (int64_t)T * r, B, D_out,
-                     idx, scale, y, ldy, y_col_off, 1, meta, meta_bytes, stream);
+  return expand_impl(dtype, T, r, S, n_slices, buf, shared_A ? 0 : (int64_t)T * r, B, D_out,
+                     idx, scale, y, ldy, y_col_off, 1, meta, meta_bytes, stream, 1);
 }
 
 int lora_bgmv_launches(lora_dtype dtype, int T, int D, int r, int S, int n_slices,

@@ -110,17 +110,6 @@ __device__ void validate_segments(const int32_t* ss, const int32_t* sa, int n_se
   if (badi) atomicAdd(bad_index, badi);
 }
 
-// The per-token grouping in the workspace was built for (T, S): otherwise its
-// positions are not known to lie in this call's buffers, so nothing is done
-// and the error is counted once (the error counters head the workspace).
-__device__ bool grouped_meta_ok(int* counters, int T, int S, bool count) {
-  const MetaHeader* h = reinterpret_cast<const MetaHeader*>(counters);
-  if (h->T == T && h->S == S) return true;
-  if (count && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
-    atomicAdd(&reinterpret_cast<MetaHeader*>(counters)->bad_meta, 1);
-  return false;
-}
-
 template <int SW>
 __device__ __forceinline__ int swz(int row, int chunk) {
   if constexpr (SW == 128) return chunk ^ (row & 7);
@@ -161,7 +150,8 @@ struct ShrinkSmem {
   static constexpr int kPitch = R + 4;                     // floats, partial-sum rows
   static constexpr int kStages = stages_for<R>();
   static constexpr size_t kBar = (size_t)kStageBytes * kStages;
-  static constexpr size_t kTotal = kBar + 8 * (2 * kStages + 1) + 64 + 1024;
+  static constexpr size_t kTok = kBar + 8 * (2 * kStages + 1) + 64;   // int [kTM]
+  static constexpr size_t kTotal = kTok + 4 * kTM + 1024;
 };
 
 static_assert(2 * (ShrinkSmem<16>::kTotal + 1024) <= 228 * 1024 &&
@@ -196,20 +186,29 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   uint64_t* accbar = empty + kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accbar + 1);
   int* sinfo = reinterpret_cast<int*>(tmem_slot + 4);
+  int* stok = reinterpret_cast<int*>(smem + L::kTok);
 
   if (blockIdx.x == 0 && slice == 0 && !P.implicit_slots)
     validate_segments(P.seg_starts, P.seg_adapter, P.n_seg, P.T, P.S, P.bad_index, P.bad_meta);
-  // grouping metadata must have been built for this call's sizes
-  const bool meta_ok = !P.implicit_slots || grouped_meta_ok(P.bad_index, P.T, P.S, tid == 0);
   if (warp == 0) {
+    // the tile is looked up while the header is read (the lookup stays inside
+    // the workspace whatever sizes it was built for); the grouping metadata
+    // must have been built for this call's sizes
+    const MetaHeader* hdr = reinterpret_cast<const MetaHeader*>(P.meta);
+    const int hT = P.implicit_slots ? hdr->T : P.T, hS = P.implicit_slots ? hdr->S : P.S;
+    const int has_ranks = hdr->has_ranks;
     TileInfo ti;
-    const bool found = meta_ok && find_tile(blockIdx.x / KS, P.seg_starts, P.seg_adapter,
-                                            P.n_seg, P.T, ti, P.implicit_slots);
+    const bool found = find_tile(blockIdx.x / KS, P.seg_starts, P.seg_adapter, P.n_seg, P.T, ti,
+                                 P.implicit_slots);
+    const bool meta_ok = hT == P.T && hS == P.S;
+    if (!meta_ok && lane == 0 && blockIdx.x == 0 && slice == 0) atomicAdd(P.bad_meta, 1);
     if (lane == 0) {
-      sinfo[0] = found ? 1 : 0;
+      sinfo[0] = found && meta_ok ? 1 : 0;
       sinfo[1] = ti.m0;
       sinfo[2] = ti.valid;
       sinfo[3] = ti.adapter;
+      // the slot's own rank (a multiple of 8, or R)
+      sinfo[4] = has_ranks && found && meta_ok ? slot_rank(P.meta, P.S, ti.adapter, R) : R;
     }
   }
   __syncthreads();
@@ -229,9 +228,13 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   };
   if (adapter < 0 || adapter >= P.S) {        // no adapter: zero rows (rank 0 writes them)
     if (kr == 0)
-      for (int e = tid; e < valid * R; e += kShrThreads) {
-        const int t = token(m0 + e / R, e % R == 0);
-        if (t >= 0) bufs[(size_t)t * R + e % R] = 0.f;
+      for (int m = tid; m < valid; m += kShrThreads) {
+        const int t = token(m0 + m, true);
+        if (t >= 0) {
+          float4* row = reinterpret_cast<float4*>(bufs + (size_t)t * R);
+#pragma unroll
+          for (int q = 0; q < R / 4; ++q) row[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
     return;
   }
@@ -241,11 +244,23 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   const int nkb = kb1 - kb0;                  // >= 1 (the host keeps KS <= nkb_all)
   // the slot's own rank kk (a multiple of 8): only its first kk rows of A are
   // read, and the MMA is N = kk rounded up to 16 wide
-  const int kk = slot_rank(P.meta, P.S, adapter, R);
+  const int kk = sinfo[4];
   const uint32_t idesc = ptx::umma_idesc_f16(kBF, kTM, kk < 16 ? 16 : (kk + 15) & ~15);
   const uint32_t a_bytes = (uint32_t)kk * 128;
 
   const int ngroups = (valid + 3) / 4;        // 4-row gathers per stage (row indirection)
+  // load warps: gather g = warp + 4 * lane brings tile rows 4g..4g+3; their
+  // tokens are the same at every K step, so they are read once, here, while
+  // the barriers and tensor memory are set up
+  const int g = warp + 4 * lane;
+  int rr[4] = {0, 0, 0, 0};
+  if (warp < 4 && perm && g < ngroups) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int p = m0 + 4 * g + j;
+      rr[j] = perm[p < m0 + valid ? p : m0];
+    }
+  }
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(&full[s], 4);           // one arrival per load warp
@@ -268,17 +283,7 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   bool ok = true;
   if (warp < 4) {
     // load warps: the adapter tile and the x tile (one 2-D tile, or up to 32
-    // four-row gathers, gather g issued by warp g % 4, lane g / 4); a gather's
-    // four token rows are the same at every K step, so they are read once
-    const int g = warp + 4 * lane;
-    int rr[4] = {0, 0, 0, 0};
-    if (perm && g < ngroups) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int p = m0 + 4 * g + j;
-        rr[j] = perm[p < m0 + valid ? p : m0];
-      }
-    }
+    // four-row gathers, gather g issued by warp g % 4, lane g / 4)
     for (int i = 0; i < nkb; ++i) {
       const int s = i % kStages;
       const uint32_t ph = (i / kStages) & 1;
@@ -305,6 +310,11 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
       if (perm && g < ngroups)
         ptx::tma_gather4(st + g * 4 * 128, &P.tmX, kx, rr[0], rr[1], rr[2], rr[3], &full[s]);
     }
+    // while the MMAs run: the token of each tile row, checked against the
+    // batch's indices, for the epilogue; a stale row is counted by the rank
+    // that writes it
+    const int m = warp * 32 + lane;
+    stok[m] = m < valid ? token(m0 + m, KS == 1 || m / ((valid + KS - 1) / KS) == kr) : -1;
   } else if (lane == 0) {
     // MMA issuer (warp 4)
     const uint32_t sbase = ptx::smem_u32(smem);
@@ -330,45 +340,57 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   const int m = warp * 32 + lane;
   float v[R];
   if (has_row) {
+    uint32_t r[R];
 #pragma unroll
-    for (int c = 0; c < R / 16; ++c) {
-      uint32_t r[16];
-      ptx::tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c * 16, r);
-      ptx::tc_wait_ld();
-      // columns past the slot's rank: zero (the accumulator holds nothing there)
+    for (int c = 0; c < R / 16; ++c) ptx::tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c * 16, r + c * 16);
+    ptx::tc_wait_ld();
+    // columns past the slot's rank: zero (the accumulator holds nothing there)
 #pragma unroll
-      for (int u = 0; u < 16; ++u) v[c * 16 + u] = c * 16 + u < kk ? __uint_as_float(r[u]) : 0.f;
-    }
+    for (int u = 0; u < R; ++u) v[u] = u < kk ? __uint_as_float(r[u]) : 0.f;
   }
   if (KS == 1) {
-    const int t = has_row && m < valid ? token(m0 + m, true) : -1;
+    const int t = has_row ? stok[m] : -1;
     if (t >= 0) {
       float4* row = reinterpret_cast<float4*>(bufs + (size_t)t * R);
 #pragma unroll
       for (int q = 0; q < R / 4; ++q) row[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
   } else {
-    // Split-K sum.  Row m belongs to rank m / rows; every rank pushes its
-    // partial row into slot [kr] of the owner's receive area (the owner's
-    // drained stage memory), then each owner adds its KS slots in rank order.
-    const int rows = kTM / KS;
+    // Split-K sum over the tile's valid rows: row m belongs to rank m / rpr;
+    // every rank pushes its partial of the row into slot [kr] of the owner's
+    // receive area (the owner's drained stage memory), then each owner adds
+    // its KS slots in rank order.
+    const int rpr = (valid + KS - 1) / KS;
     cluster.barrier_arrive();                 // this CTA's MMAs and stages are done...
     cluster.barrier_wait();                   // ...and so are every peer's
     float* recv = reinterpret_cast<float*>(smem);
-    if (has_row) {
-      float* dst = cluster.map_shared_rank(recv, m / rows) + (size_t)(kr * rows + m % rows) * L::kPitch;
+    if (has_row && m < valid) {
+      float* dst = cluster.map_shared_rank(recv, m / rpr) + (size_t)(kr * rpr + m % rpr) * L::kPitch;
 #pragma unroll
       for (int q = 0; q < R / 4; ++q)
         reinterpret_cast<float4*>(dst)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
     cluster.sync();                           // every partial has arrived
-    for (int e = tid; e < rows * R; e += kShrThreads) {
-      const int lm = e / R, j = e % R;
-      float sum = 0.f;
-      for (int q = 0; q < KS; ++q) sum += recv[(size_t)(q * rows + lm) * L::kPitch + j];
-      const int mm = kr * rows + lm;
-      const int t = mm < valid ? token(m0 + mm, j == 0) : -1;
-      if (t >= 0) bufs[(size_t)t * R + j] = sum;
+    // four columns of an owned row per step, every partial loaded first
+    const int own0 = kr * rpr, nown = max(0, min(rpr, valid - own0));
+    const float4* rv = reinterpret_cast<const float4*>(recv);
+    for (int e = tid; e < nown * (R / 4); e += kShrThreads) {
+      const int lm = e / (R / 4), c = e % (R / 4);
+      float4 part[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (q < KS) part[q] = rv[(size_t)(q * rpr + lm) * (L::kPitch / 4) + c];
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (q < KS) {
+          sum.x += part[q].x;
+          sum.y += part[q].y;
+          sum.z += part[q].z;
+          sum.w += part[q].w;
+        }
+      const int t = stok[own0 + lm];
+      if (t >= 0) reinterpret_cast<float4*>(bufs + (size_t)t * R)[c] = sum;
     }
   }
   ptx::tc_fence_before();
@@ -386,13 +408,15 @@ struct SegView {
   const int32_t* sa;
   int n_seg, T, S, implicit_slots;
   int4* cache;                           // shared-memory copy of the first kSegCache segments
-  // the same, from the copy when the whole list is in it
-  __device__ __forceinline__ void get_cached(int s, int& a, int& b, int& ad) const {
+  // the same, from the copy when the whole list is in it; kc = the adapter's
+  // rank class from the copy, or -1 when it is not cached
+  __device__ __forceinline__ void get_cached(int s, int& a, int& b, int& ad, int& kc) const {
     if (n_seg <= kSegCache) {
       const int4 c = s < n_seg ? cache[s] : make_int4(0, 0, -1, 0);
-      a = c.x; b = c.y; ad = c.z;
+      a = c.x; b = c.y; ad = c.z; kc = c.w;
     } else {
       get(s, a, b, ad);
+      kc = -1;
     }
   }
   // segment s clamped into [0, T]; adapter -1 when it has none or is out of range
@@ -458,6 +482,7 @@ struct ExpandTCParams {
   int* bad_index;
   int* bad_meta;
   const char* meta;                      // workspace: per-slot ranks
+  int early;                             // wait for the previous kernel only before reading buf
 };
 
 template <int R>
@@ -502,10 +527,21 @@ __device__ __forceinline__ int64_t seg_weight(int a, int b, int ad) {
   return (int64_t)(len / kTM) * pair_weight<R>(kTM) + (rem ? pair_weight<R>(rem) : 0);
 }
 
-// Warp 0 of the CTA: per-chunk (32 segments) weights into chunkW, total
-// returned in every lane.
+// Rank class of an adapter: its rank rounded up to 16 << kc (the call's rank
+// when the workspace holds no per-slot ranks; nothing is read then).
 template <int R>
-__device__ int64_t seg_chunk_weights(const SegView& sv, int64_t* chunkW) {
+__device__ __forceinline__ int rank_class(const char* meta, int S, int adapter, int has_ranks) {
+  const int k = has_ranks ? slot_rank(meta, S, adapter, R) : R;
+  const int k16 = max(16, (k + 15) & ~15);
+  return k16 == 16 ? 0 : (k16 == 32 ? 1 : 2);
+}
+
+// Warp 0 of the CTA: per-chunk (32 segments) weights into chunkW, total
+// returned in every lane; the first kSegCache segments and their adapters'
+// rank classes are copied to shared memory.
+template <int R>
+__device__ int64_t seg_chunk_weights(const SegView& sv, int64_t* chunkW, const char* meta,
+                                     int has_ranks) {
   const int lane = threadIdx.x & 31;
   const int nch = (sv.n_seg + 31) / 32;
   int64_t total = 0;
@@ -516,7 +552,8 @@ __device__ int64_t seg_chunk_weights(const SegView& sv, int64_t* chunkW) {
       int a, b, ad;
       const int sidx = (c0 + u) * 32 + lane;
       sv.get(sidx, a, b, ad);
-      if (sidx < kSegCache) sv.cache[sidx] = make_int4(a, b, ad, 0);
+      if (sidx < kSegCache)
+        sv.cache[sidx] = make_int4(a, b, ad, ad >= 0 ? rank_class<R>(meta, sv.S, ad, has_ranks) : 0);
       w[u] = seg_weight<R>(a, b, ad);
     }
 #pragma unroll
@@ -535,17 +572,10 @@ __device__ int64_t seg_chunk_weights(const SegView& sv, int64_t* chunkW) {
 // Warp-cooperative: the tile runs whose pair start positions fall in
 // [lo, hi), in schedule order, at most kMaxRuns of them.  Returns the count;
 // *next is hi when the list is complete, else where the next list starts.
-// Rank class of an adapter: its rank rounded up to 16 << kc.
-template <int R>
-__device__ __forceinline__ int rank_class(const char* meta, int S, int adapter) {
-  const int k16 = max(16, (slot_rank(meta, S, adapter, R) + 15) & ~15);
-  return k16 == 16 ? 0 : (k16 == 32 ? 1 : 2);
-}
-
 template <int R>
 __device__ int build_runs(const SegView& sv, const int64_t* chunkW, int64_t Wt,
                           const int* ntiles, int n_slices, int64_t lo, int64_t hi,
-                          ExpRun* runs, int64_t* next, const char* meta) {
+                          ExpRun* runs, int64_t* next, const char* meta, int has_ranks) {
   const int lane = threadIdx.x & 31;
   const int nch = (sv.n_seg + 31) / 32;
   int n = 0;
@@ -564,8 +594,8 @@ __device__ int build_runs(const SegView& sv, const int64_t* chunkW, int64_t Wt,
         cpos += cw;
         continue;
       }
-      int a, b, ad;
-      sv.get_cached(c * 32 + lane, a, b, ad);
+      int a, b, ad, kc;
+      sv.get_cached(c * 32 + lane, a, b, ad, kc);
       const int64_t sw = nt * seg_weight<R>(a, b, ad);
       int64_t incl = sw;
 #pragma unroll
@@ -582,7 +612,8 @@ __device__ int build_runs(const SegView& sv, const int64_t* chunkW, int64_t Wt,
         const int len = __shfl_sync(0xffffffffu, b, l) - a_l;
         const int ad_l = __shfl_sync(0xffffffffu, ad, l);
         const int64_t sp = __shfl_sync(0xffffffffu, spos, l);
-        const int kc_l = rank_class<R>(meta, sv.S, ad_l);
+        const int kc_c = __shfl_sync(0xffffffffu, kc, l);
+        const int kc_l = kc_c >= 0 ? kc_c : rank_class<R>(meta, sv.S, ad_l, has_ranks);
         const int ntk = (len + kTM - 1) / kTM;
         for (int k0 = 0; k0 < ntk; k0 += 32) {
           const int k = k0 + lane;
@@ -626,7 +657,11 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   constexpr int kYS = L::kYS;
   constexpr bool kBF = std::is_same<E, __nv_bfloat16>::value;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  ptx::grid_dep_wait();               // grouping, buf and y producers have finished
+  // The previous kernel (programmatic dependent launch) is waited for here,
+  // or, when it is known to be the shrink of the same batch, only by the load
+  // warps before their first buf read: the run lists, the B tiles and the y
+  // tiles of the first pairs are then set up while the shrink finishes.
+  if (!P.early) ptx::grid_dep_wait();
   ptx::grid_dep_launch_dependents();
 
   extern __shared__ char smem_raw[];
@@ -661,13 +696,19 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
     sum_nt += ntiles[i];
   }
 
+  int has_ranks = 0;                     // read by the MMA warp, which builds the run lists
   if (warp == kExpMma) {
     ptx::tmem_alloc(tmem_slot, 2 * kNT);
     ptx::tmem_relinquish();
     // this CTA's share of the weighted pair sequence (the segment reads stay in
-    // bounds whatever the workspace holds, so they need not wait for the check)
-    const int64_t Wt0 = seg_chunk_weights<R>(sv, chunkW);
-    const bool meta_ok = !P.implicit_slots || grouped_meta_ok(P.bad_index, P.T, P.S, lane == 0);
+    // bounds whatever the workspace holds, so they are made while the header
+    // is read)
+    const MetaHeader* hdr = reinterpret_cast<const MetaHeader*>(P.meta);
+    const int hT = P.implicit_slots ? hdr->T : P.T, hS = P.implicit_slots ? hdr->S : P.S;
+    has_ranks = hdr->has_ranks;
+    const int64_t Wt0 = seg_chunk_weights<R>(sv, chunkW, P.meta, has_ranks);
+    const bool meta_ok = hT == P.T && hS == P.S;
+    if (!meta_ok && lane == 0 && blockIdx.x == 0) atomicAdd(P.bad_meta, 1);
     const int64_t Wt = meta_ok ? Wt0 : 0;
     const int64_t W = Wt * sum_nt;
     if (lane == 0) {
@@ -706,7 +747,8 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   while (lo < hi) {
     if (warp == kExpMma) {
       int64_t nx;
-      const int n = build_runs<R>(sv, chunkW, Wt, ntiles, P.n_slices, lo, hi, runs, &nx, P.meta);
+      const int n = build_runs<R>(sv, chunkW, Wt, ntiles, P.n_slices, lo, hi, runs, &nx, P.meta,
+                                  has_ranks);
       if (lane == 0) {
         *sNRuns = n;
         sRange[3] = nx;
@@ -721,6 +763,7 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
       const int pw = warp - kExpLoad0;
       const int lt = pw * 32 + lane;                 // operand row of this thread
       int pl = p, ul = u;
+      bool buf_ready = !P.early;
       for (int ri = 0; ri < n_runs; ++ri, ++ul) {
         const ExpRun rn = runs[ri];
         const int hb = ul & 1;
@@ -732,12 +775,10 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
         const int m = lt;
         // sTok: the row's token; -1 past the tile; -2 - token for a token whose
         // index disagrees with its group (stale workspace): still a valid row
-        // address for the gathers, but never written back (counted here)
-        int tok = m < rn.valid ? (P.perm ? P.perm[rn.m0 + m] : rn.m0 + m) : -1;
-        if (tok >= 0 && P.perm && !grouped_row_ok(P.idx, tok, rn.adapter, P.S)) {
-          if (rn.j0 == 0) atomicAdd(P.bad_meta, 1);
-          tok = -2 - tok;
-        }
+        // address for the gathers, but never written back (counted below).
+        // The gathers need only the token, so the index check is made after
+        // they are issued, together with the buf row read.
+        const int tok = m < rn.valid ? (P.perm ? P.perm[rn.m0 + m] : rn.m0 + m) : -1;
         sTok[hb * kTM + m] = tok;
         asm volatile("bar.sync 4, 128;" ::: "memory");   // every row's token is known
         const int* toks = sTok + hb * kTM;
@@ -790,8 +831,13 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
         // hi / lo after an exact power-of-two rescale 2^(7-e) (e = exponent of
         // the row's max |buf|), and the inverse scale
         {
+          if (!buf_ready) {
+            ptx::grid_dep_wait();                    // the shrink has written buf
+            buf_ready = true;
+          }
           const float4* brow = reinterpret_cast<const float4*>(
               P.buf + (size_t)rn.slice * P.buf_slice_stride + (size_t)(tok < 0 ? 0 : tok) * R);
+          const bool stale = tok >= 0 && P.perm && !grouped_row_ok(P.idx, tok, rn.adapter, P.S);
           float4 f[R / 4];
           float mx = 0.f;
 #pragma unroll
@@ -821,6 +867,10 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
             *reinterpret_cast<uint4*>(loP + off) = *reinterpret_cast<const uint4*>(l8);
           }
           sInv[hb * kTM + m] = __int_as_float((127 + e - 7) << 23);
+          if (stale) {
+            if (rn.j0 == 0) atomicAdd(P.bad_meta, 1);
+            sTok[hb * kTM + m] = -2 - tok;   // the gathers read either form as row tok
+          }
           ptx::fence_proxy_async_smem();   // generic writes -> tensor-core operand reads
         }
         __syncwarp();
@@ -1194,6 +1244,7 @@ cudaError_t expand_tc_launch(const ExpandArgs& a, const SegArgs& sg, lora_dtype 
   P.bad_index = const_cast<int*>(&hdr->bad_index);
   P.bad_meta = const_cast<int*>(&hdr->bad_meta);
   P.meta = a.meta;
+  P.early = a.after_shrink;
   // one CTA per SM, never more CTAs than (tile, n-tile) pairs
   const long max_tiles = (a.T + kTM - 1) / kTM + sg.n_seg;
   const long pairs = max_tiles * sum_nt;
