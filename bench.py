@@ -867,6 +867,17 @@ def laning_block(stream, peak, reps=256):
     return out
 
 
+def pick_workload(args):
+    ps = W.config(args.config)
+    if args.workload is None:
+        return ps[0]
+    for p in ps:
+        if p.name == args.workload:
+            return p
+    raise SystemExit(f"config {args.config} has no workload {args.workload!r} "
+                     f"(it has {', '.join(q.name for q in ps)})")
+
+
 def run_ours(args):
     ws, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -875,7 +886,7 @@ def run_ours(args):
     from gather_matmul_b200 import ops
     ops.build_info()   # loads the library or fails loudly
 
-    p = W.config(args.config)[0]
+    p = pick_workload(args)
     if rank:   # data parallel: every rank serves its own batch of the same shape
         p = W.make_problem(p.name, p.dtype, p.T, p.D, p.r, p.S, p.d_out, p.scale,
                            seed=1000 * rank + args.config,
@@ -970,7 +981,7 @@ def run_reference(args):
     if rank != 0:
         return
     import oracle
-    p = W.config(args.config)[0]
+    p = pick_workload(args)
     cores = oracle.set_threads(os.cpu_count() or 1)
     idx = p.idx if not p.segmented else oracle.segments_to_idx(p.T, p.seg_starts, p.seg_adapter)
     shared = p.shared_A and p.n_slices > 1
@@ -1019,6 +1030,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", type=int, default=5, choices=[1, 2, 3, 4, 5],
                     help="headline workload (default 5: the large mixed batch)")
+    ap.add_argument("--workload", default=None,
+                    help="one workload of the config by name (default: its first), e.g. "
+                         "decode_gate_up of config 3")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-configs", action="store_true",
                     help="leave out the per-workload block")

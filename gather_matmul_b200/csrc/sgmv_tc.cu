@@ -510,12 +510,21 @@ struct ExpandSmem {
   static_assert(kOffChunk % 8 == 0 && kOffSeg % 16 == 0 && kOffBar % 8 == 0, "alignment");
 };
 
-// Bytes a pair moves, in units the schedule balances: the B tile, the valid
-// y rows read and written, and a fixed per-pair cost (the pipeline time of a
-// pair that moves almost nothing, in bytes at one SM's share of HBM bandwidth).
+// The time a pair takes on one SM, in quarter nanoseconds, as measured on
+// B200 by a least-squares fit of each CTA's time against its pairs and rows
+// (Zipf, uniform and mixed-size batches at rank 32):
+//   operand-swapped tile (<= 64 rows): 0.58 us + 16.5 ns per valid row: its
+//     epilogue is one round of the pipeline for few rows;
+//   128-row layout (65..128 rows): 1.2 us + 5 ns per valid row, nearly flat:
+//     the whole tile passes through tensor memory and the epilogue;
+//   plus about 4.5 ns per rank column of the B tile (its 256 r bytes).
+// Weights in bytes moved rated a full tile at 3.3 small tiles (it costs
+// about 2.8) and a 90-row tile far below a full one (it costs 90 %), which
+// left CTAs of small groups as the long poles.
 template <int R>
 __device__ __forceinline__ int64_t pair_weight(int valid) {
-  return (int64_t)kNT * R * 2 + 512 * (int64_t)valid + 16384;
+  return valid <= kSwapMax ? 1744 + 18 * R + 66 * (int64_t)valid
+                           : 4224 + 18 * R + 20 * (int64_t)valid;
 }
 
 // Per n-tile weight of one segment: its full tiles and its partial last tile.
