@@ -619,6 +619,37 @@ def workload_numbers(p, t_step, kt, peak, tf_peak, fused_fits, launches):
     }
 
 
+def copy_floor(nbytes, stream, reps=256):
+    """Device time of ONE plain copy kernel (torch's) that reads nbytes / 2 and
+    writes nbytes / 2, timed like the steps (graph replay over rotating buffers
+    larger than L2): the speed a single launch moving the step's bytes reaches
+    at this size, launch and ramp included.  A reference for the fractions,
+    not part of the path."""
+    half = max(4096, (nbytes // 2) // 4096 * 4096)
+    n = rotation_sets(2 * half)
+    bufs = [(torch.ones(half, dtype=torch.uint8, device="cuda"),
+             torch.empty(half, dtype=torch.uint8, device="cuda")) for _ in range(n)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for k in range(reps):
+            src, dst = bufs[k % n]
+            dst.copy_(src)
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / reps
+    del g, bufs
+    torch.cuda.empty_cache()
+    return t, 2 * half
+
+
 def measure_workload(p, stream, reps, peak, tf_peak):
     sets = make_sets(p)
     ff = fused(p)
@@ -629,6 +660,11 @@ def measure_workload(p, stream, reps, peak, tf_peak):
     out["l2"] = f"{len(sets)} rotating input sets, {sum(s.nbytes() for s in sets) / 1e6:.0f} MB"
     del sets
     torch.cuda.empty_cache()
+    tc, cb = copy_floor(algorithmic_bytes(p)["step"], stream, reps)
+    out["one_launch_copy"] = {"bytes": cb, "us": round(tc * 1e6, 3),
+                              "gbs": round(cb / tc / 1e9, 1),
+                              "frac_hbm": round(cb / tc / 1e9 / peak, 4),
+                              "step_time_ratio": round(tc / t, 4)}
     return out
 
 
