@@ -56,6 +56,63 @@ __device__ int block_exclusive_scan(int* a, int n, int* warp_tmp) {
   return total;
 }
 
+// Exclusive scans of two arrays of n <= 2 * kGroupThreads ints in shared
+// memory, in place, sharing their barriers; the totals go to *ta and *tb.
+// Must be called by all threads of the block.
+__device__ void block_exclusive_scan2(int* a, int* b, int n, int* warp_tmp, int* ta, int* tb) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int i0 = 2 * tid, i1 = 2 * tid + 1;
+  const int a0 = i0 < n ? a[i0] : 0, a1 = i1 < n ? a[i1] : 0;
+  const int b0 = i0 < n ? b[i0] : 0, b1 = i1 < n ? b[i1] : 0;
+  const int sa = a0 + a1, sb = b0 + b1;
+  int ia = sa, ib = sb;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int ua = __shfl_up_sync(0xffffffffu, ia, o);
+    const int ub = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) {
+      ia += ua;
+      ib += ub;
+    }
+  }
+  if (lane == 31) {
+    warp_tmp[warp] = ia;
+    warp_tmp[32 + warp] = ib;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int wa = lane < kGroupWarps ? warp_tmp[lane] : 0;
+    const int wb = lane < kGroupWarps ? warp_tmp[32 + lane] : 0;
+    int xa = wa, xb = wb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ua = __shfl_up_sync(0xffffffffu, xa, o);
+      const int ub = __shfl_up_sync(0xffffffffu, xb, o);
+      if (lane >= o) {
+        xa += ua;
+        xb += ub;
+      }
+    }
+    warp_tmp[64 + lane] = xa - wa;     // exclusive prefixes of the warp totals
+    warp_tmp[96 + lane] = xb - wb;
+    if (lane == 31) {
+      *ta = xa;
+      *tb = xb;
+    }
+  }
+  __syncthreads();
+  const int ea = warp_tmp[64 + warp] + ia - sa, eb = warp_tmp[96 + warp] + ib - sb;
+  if (i0 < n) {
+    a[i0] = ea;
+    b[i0] = eb;
+  }
+  if (i1 < n) {
+    a[i1] = ea + a0;
+    b[i1] = eb + b0;
+  }
+  __syncthreads();
+}
+
 // Generation barrier of the grouping kernel's CTAs, kept in the workspace
 // header.  Thread 0 of each CTA calls it once its CTA's histogram row is
 // written and fenced.  The last CTA to arrive resets the count and opens the
@@ -86,29 +143,36 @@ __device__ bool group_barrier(MetaHeader* hdr, int nb) {
 
 constexpr int kLoadBatch = 8;   // indices a lane has in flight at once
 
+// Per-(key, warp) counts are kept key-major with a pitch of 33 ints, so the
+// counts of one key across the 32 warps are one conflict-free row that a
+// warp scans with shuffles.
+constexpr int kCntPitch = kGroupWarps + 1;
+
 // group_ctas(T) CTAs, each over a contiguous chunk of the tokens; each warp
 // over a contiguous part of its CTA's chunk, so CTA, warp and lane order is
-// token order and the scatter is stable.  Shared memory: cnt[kGroupWarps][K],
-// tot[K], base[K], pre[K], ni[K] and 66 ints of scan scratch, K = S + 1 keys
-// (key S = no adapter).
-//   1. per-warp counts of each key (warp match_any), summed into this CTA's
-//      row of the workspace histogram;
+// token order and the scatter is stable.  Shared memory: cnt[K][33],
+// tot[K], base[K], pre[K], ni[K] and 130 ints of scan scratch, K = S + 1
+// keys (key S = no adapter).
+//   1. per-warp counts of each key (warp match_any); one warp per key scans
+//      the key's 32 warp counts (each warp's offset inside the CTA) and
+//      writes the CTA's total into its row of the workspace histogram;
 //   2. barrier over the CTAs;
 //   3. every CTA reads the histogram: each key's total and the part of it in
-//      earlier CTAs; block scans give each key's first position and the work
-//      list offsets;
-//   4. stable scatter of this CTA's tokens into perm; CTA 0 writes the slot
-//      offsets and header, the work items are shared out by key.
+//      earlier CTAs; one pair of block scans gives each key's first position
+//      and the work list offsets;
+//   4. stable scatter of this CTA's tokens into perm (a warp's first batch of
+//      indices is still in registers); CTA 0 writes the slot offsets and
+//      header, the work items are shared out by key.
 __global__ void __launch_bounds__(kGroupThreads, 1)
 group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ meta) {
   extern __shared__ int smem[];
   const int K = S + 1;
-  int* cnt = smem;                          // [warp][key]
-  int* tot = cnt + kGroupWarps * K;         // this CTA's count, then the total, per key
+  int* cnt = smem;                          // [key][kCntPitch]
+  int* tot = cnt + K * kCntPitch;           // this CTA's count, then the total, per key
   int* base = tot + K;                      // first position per key
   int* pre = base + K;                      // tokens of the key in earlier CTAs
   int* ni = pre + K;                        // items per key, then item offsets
-  int* scratch = ni + K;                    // 65 ints of scan scratch + a flag
+  int* scratch = ni + K;                    // 128 ints of scan scratch, 2 totals, a flag
 
   ptx::grid_dep_wait();               // the previous kernel's writes (idx, meta) are visible
   ptx::grid_dep_launch_dependents();
@@ -127,9 +191,12 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
   const int beg = min(c1, c0 + warp * wchunk);
   const int end = min(c1, beg + wchunk);
 
-  for (int i = tid; i < kGroupWarps * K; i += kGroupThreads) cnt[i] = 0;
+  for (int i = tid; i < K * kCntPitch; i += kGroupThreads) cnt[i] = 0;
   __syncthreads();
 
+  // a warp's first batch of indices stays in registers for the scatter pass
+  // (the only batch while a warp's part is at most 32 * kLoadBatch tokens)
+  int v0[kLoadBatch];
   int bad = 0;
   for (int b0 = beg; b0 < end; b0 += 32 * kLoadBatch) {
     int v[kLoadBatch];
@@ -137,6 +204,10 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
     for (int u = 0; u < kLoadBatch; ++u) {
       const int t = b0 + 32 * u + lane;
       v[u] = t < end ? __ldg(idx + t) : -1;
+    }
+    if (b0 == beg) {
+#pragma unroll
+      for (int u = 0; u < kLoadBatch; ++u) v0[u] = v[u];
     }
 #pragma unroll
     for (int u = 0; u < kLoadBatch; ++u) {
@@ -146,7 +217,7 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
       if (valid && (v[u] < -1 || v[u] >= S)) ++bad;
       const int key = valid ? ((v[u] >= 0 && v[u] < S) ? v[u] : S) : -1;
       const unsigned peers = __match_any_sync(0xffffffffu, key);
-      if (valid && lane == __ffs(peers) - 1) cnt[warp * K + key] += __popc(peers);
+      if (valid && lane == __ffs(peers) - 1) cnt[key * kCntPitch + warp] += __popc(peers);
     }
   }
 #pragma unroll
@@ -154,20 +225,28 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
   if (lane == 0 && bad) atomicAdd(&hdr->bad_index, bad);
   __syncthreads();
 
-  for (int k = tid; k < K; k += kGroupThreads) {
-    int c = 0;
-    for (int w = 0; w < kGroupWarps; ++w) c += cnt[w * K + k];
-    tot[k] = c;
-    if (nb > 1) {
-      hist[cta * K + k] = c;
-      __threadfence();
+  // key k, lane = warp w: the warp's offset among the CTA's tokens of key k,
+  // and the CTA's total of key k
+  for (int k = warp; k < K; k += kGroupWarps) {
+    const int c = cnt[k * kCntPitch + lane];
+    int inc = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += u;
+    }
+    cnt[k * kCntPitch + lane] = inc - c;
+    if (lane == 31) {
+      tot[k] = inc;
+      if (nb > 1) hist[cta * K + k] = inc;
     }
   }
+  if (nb > 1) __threadfence();
   __syncthreads();
   if (nb > 1) {
-    if (tid == 0) scratch[65] = group_barrier(hdr, nb) ? 1 : 0;
+    if (tid == 0) scratch[130] = group_barrier(hdr, nb) ? 1 : 0;
     __syncthreads();
-    if (!scratch[65]) {                           // another CTA never arrived
+    if (!scratch[130]) {                          // another CTA never arrived
       if (tid == 0) atomicAdd(&hdr->bad_meta, 1);
       return;
     }
@@ -187,16 +266,15 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
   }
   __syncthreads();
   // K <= LORA_MAX_SLOTS + 1 <= 2 * kGroupThreads
-  block_exclusive_scan(base, K, scratch);
-  const int n_items = block_exclusive_scan(ni, K, scratch);
+  block_exclusive_scan2(base, ni, K, scratch, scratch + 128, scratch + 129);
+  const int n_items = scratch[129];
 
+  // per-(key, warp) start positions
+  for (int e = tid; e < K * kGroupWarps; e += kGroupThreads) {
+    const int k = e / kGroupWarps, w = e % kGroupWarps;
+    cnt[k * kCntPitch + w] += base[k] + pre[k];
+  }
   for (int k = tid; k < K; k += kGroupThreads) {
-    int run = base[k] + pre[k];
-    for (int w = 0; w < kGroupWarps; ++w) {   // per-(warp, key) start positions
-      const int c = cnt[w * K + k];
-      cnt[w * K + k] = run;
-      run += c;
-    }
     if (cta == 0) slot_off[k] = base[k];
     if (k % nb == cta) {
       const int it0 = ni[k], n = tot[k];
@@ -223,7 +301,7 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
 #pragma unroll
     for (int u = 0; u < kLoadBatch; ++u) {
       const int t = b0 + 32 * u + lane;
-      v[u] = t < end ? __ldg(idx + t) : -1;
+      v[u] = b0 == beg ? v0[u] : (t < end ? __ldg(idx + t) : -1);
     }
 #pragma unroll
     for (int u = 0; u < kLoadBatch; ++u) {
@@ -233,11 +311,11 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
       const int key = valid ? ((v[u] >= 0 && v[u] < S) ? v[u] : S) : -1;
       const unsigned peers = __match_any_sync(0xffffffffu, key);
       int pos = 0;
-      if (valid) pos = cnt[warp * K + key] + __popc(peers & lanemask_lt());
+      if (valid) pos = cnt[key * kCntPitch + warp] + __popc(peers & lanemask_lt());
       __syncwarp();
       if (valid) {
         perm[pos] = t;
-        if (lane == __ffs(peers) - 1) cnt[warp * K + key] += __popc(peers);
+        if (lane == __ffs(peers) - 1) cnt[key * kCntPitch + warp] += __popc(peers);
       }
       __syncwarp();
     }
@@ -331,7 +409,7 @@ cudaError_t launch_set_ranks(int S, const int32_t* ranks, void* meta, cudaStream
 }
 
 size_t group_smem_bytes(int S) {
-  return sizeof(int) * ((size_t)(kGroupWarps + 4) * (S + 1) + 66);
+  return sizeof(int) * ((size_t)(kCntPitch + 4) * (S + 1) + 131);
 }
 
 cudaError_t launch_group(int T, int S, const int32_t* idx, void* meta, cudaStream_t st) {
