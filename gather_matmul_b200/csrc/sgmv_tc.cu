@@ -431,8 +431,13 @@ struct SegView {
   }
 };
 
-__device__ __forceinline__ int64_t ceil_pos(int64_t num, int64_t w) {
-  return num <= 0 ? 0 : (num + w - 1) / w;
+// min(ceil(num / w), nt) for a pair weight w: 32-bit arithmetic once the
+// quotient is known to be below nt (nt * w stays far below 2^32), instead of
+// a 64-bit division
+__device__ __forceinline__ int ceil_pos_nt(int64_t num, int w, int nt) {
+  if (num <= 0) return 0;
+  if (num >= (int64_t)nt * w) return nt;
+  return (int)(((uint32_t)num + (uint32_t)w - 1u) / (uint32_t)w);
 }
 
 // ---------------------------------------------------------------- expand
@@ -554,10 +559,12 @@ __device__ int64_t seg_chunk_weights(const SegView& sv, int64_t* chunkW, const c
   const int lane = threadIdx.x & 31;
   const int nch = (sv.n_seg + 31) / 32;
   int64_t total = 0;
-  for (int c0 = 0; c0 < nch; c0 += 4) {
-    int64_t w[4];
+  // four chunks per round: all their loads first, then the reductions
+  constexpr int kU = 4;
+  for (int c0 = 0; c0 < nch; c0 += kU) {
+    int64_t w[kU];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {          // all loads first, then the reductions
+    for (int u = 0; u < kU; ++u) {
       int a, b, ad;
       const int sidx = (c0 + u) * 32 + lane;
       sv.get(sidx, a, b, ad);
@@ -566,7 +573,7 @@ __device__ int64_t seg_chunk_weights(const SegView& sv, int64_t* chunkW, const c
       w[u] = seg_weight<R>(a, b, ad);
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kU; ++u) {
       int64_t v = w[u];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -627,10 +634,10 @@ __device__ int build_runs(const SegView& sv, const int64_t* chunkW, int64_t Wt,
         for (int k0 = 0; k0 < ntk; k0 += 32) {
           const int k = k0 + lane;
           const int valid = k < ntk ? min(kTM, len - k * kTM) : 0;
-          const int64_t w = pair_weight<R>(valid);
+          const int w = (int)pair_weight<R>(valid);
           const int64_t tpos = sp + nt * (int64_t)k * pair_weight<R>(kTM);
-          const int jl = (int)(ceil_pos(lo - tpos, w) < nt ? ceil_pos(lo - tpos, w) : nt);
-          const int jh = (int)(ceil_pos(hi - tpos, w) < nt ? ceil_pos(hi - tpos, w) : nt);
+          const int jl = ceil_pos_nt(lo - tpos, w, (int)nt);
+          const int jh = ceil_pos_nt(hi - tpos, w, (int)nt);
           const bool has = k < ntk && jl < jh;
           const unsigned hm = __ballot_sync(0xffffffffu, has);
           const int rank = __popc(hm & ((1u << lane) - 1));
