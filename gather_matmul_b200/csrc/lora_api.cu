@@ -409,7 +409,7 @@ namespace {
 
 // Sized for LORA_NOALLOC_MAX_TOKENS tokens over LORA_MAX_SLOTS slots; every
 // GPU that loads the library holds it until the process exits.
-constexpr size_t kNoallocScratchBytes = 197632;
+constexpr size_t kNoallocScratchBytes = 246784;
 static_assert(kNoallocScratchBytes == LORA_NOALLOC_SCRATCH_BYTES, "header and library agree");
 static __device__ __align__(256) char g_noalloc_scratch[kNoallocScratchBytes];
 

@@ -322,7 +322,7 @@ LORA_API lora_status lora_check_errors(void* meta, size_t meta_bytes, lora_strea
  *   the error counter).
  */
 #define LORA_NOALLOC_MAX_TOKENS 8192
-#define LORA_NOALLOC_SCRATCH_BYTES 197632
+#define LORA_NOALLOC_SCRATCH_BYTES 246784
 LORA_API lora_status lora_shrink_noalloc(lora_dtype dtype, int T, int D, int r, int S,
                                          int n_slices, const void* x, int64_t ldx,
                                          const void* const* A, const int32_t* idx, float* buf,

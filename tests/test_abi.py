@@ -55,14 +55,14 @@ def a256(v):
 def test_workspace_bytes_formula(L, T, S):
     tt = max(T, 1)
     max_items = T // 16 + max(S + 1, T + 1) + 2
-    ctas = min(64, max(1, -(-T // 2048)))     # grouping CTAs, one per 2048 tokens
+    ctas = min(64, max(1, -(-T // 512)))      # grouping CTAs, one per 512 tokens
     want = (256 + a256(4 * (S + 2)) + a256(4 * S) + a256(4 * tt) + a256(16 * max_items)
             + a256(4 * ctas * (S + 1)))
     assert L.lora_workspace_bytes(T, S) == want
 
 
 def test_noalloc_array_holds_the_largest_workspace(L):
-    assert L.lora_workspace_bytes(_lib.LORA_NOALLOC_MAX_TOKENS, _lib.LORA_MAX_SLOTS) <= 197632
+    assert L.lora_workspace_bytes(_lib.LORA_NOALLOC_MAX_TOKENS, _lib.LORA_MAX_SLOTS) <= 246784
 
 
 def test_workspace_bytes_rejects_out_of_range(L):
