@@ -24,7 +24,7 @@
 //   (slice, tile, 128-column) pairs (see the expand section below).  The fp32
 //   intermediate enters the tensor core as hi + lo of the input type after an
 //   exact power-of-two rescale per row (about 16 bits for bf16, 22 for fp16),
-//   two MMAs per K step into one fp32 accumulator; a tile of at most 64 rows
+//   two MMAs per K step into one fp32 accumulator; a tile of at most 48 rows
 //   swaps the operands.  y tiles move by 2-D TMA (consecutive rows) or 4-row
 //   gathers; the epilogue adds scale * acc with one round-to-nearest-even.
 //   Rows past the segment and rows without an adapter are never written.
@@ -451,7 +451,7 @@ __device__ __forceinline__ int ceil_pos_nt(int64_t num, int w, int nt) {
 //   load warps   B tile + y tile of each pair into a ring of stages; the
 //                hi / lo operand of each run (double-buffered)
 //   MMA warp     acc = hi . B^T + lo . B^T into one of two TMEM accumulators;
-//                a tile of <= 64 rows swaps the operands (M = 128 output
+//                a tile of <= kSwapMax rows swaps the operands (M = 128 output
 //                columns, N = its rows rounded to 16) so the epilogue only
 //                touches the rows that exist
 //   epilogue     y += scale * acc, one rounding; two warps per TMEM lane
@@ -461,7 +461,10 @@ struct ExpRun {
   int kc;        // the adapter's rank rounded up to 16 << kc (per-slot ranks)
 };
 constexpr int kMaxRuns = 64;
-constexpr int kSwapMax = 64;             // tiles of at most this many rows swap operands
+// tiles of at most this many rows swap operands: by the measured pair costs
+// below the two layouts break even near 54 rows (48: large mixed step 114.3 us
+// against 114.8 with 64)
+constexpr int kSwapMax = 48;
 
 struct ExpandTCParams {
   // B_i as [S*D_out_i rows, r cols], box {16 << c, 128} with a (32 << c)-byte
@@ -518,9 +521,9 @@ struct ExpandSmem {
 // The time a pair takes on one SM, in quarter nanoseconds, as measured on
 // B200 by a least-squares fit of each CTA's time against its pairs and rows
 // (Zipf, uniform and mixed-size batches at rank 32):
-//   operand-swapped tile (<= 64 rows): 0.58 us + 16.5 ns per valid row: its
-//     epilogue is one round of the pipeline for few rows;
-//   128-row layout (65..128 rows): 1.2 us + 5 ns per valid row, nearly flat:
+//   operand-swapped tile (<= kSwapMax rows): 0.58 us + 16.5 ns per valid
+//     row: its epilogue is one round of the pipeline for few rows;
+//   128-row layout (more rows): 1.2 us + 5 ns per valid row, nearly flat:
 //     the whole tile passes through tensor memory and the epilogue;
 //   plus about 4.5 ns per rank column of the B tile (its 256 r bytes).
 // Weights in bytes moved rated a full tile at 3.3 small tiles (it costs

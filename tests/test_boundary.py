@@ -213,9 +213,9 @@ def test_integer_inputs_match_oracle_bitwise(dt, D, r):
                               "bf16-full-tiles", "f16-many-slots", "bf16-many-slots"])
 def test_integer_inputs_grouped_tensor_cores_bitwise(dt, D, T, S):
     # T >= 16 S with r = 16: the per-token batch runs through the grouping on
-    # the tcgen05 kernels (groups of about 50 rows take the operand-swapped
-    # expand, about 100 rows the full 128-row tile, about 20 rows the
-    # swapped tile with few rows).  x, A, B in {-1,0,1},
+    # the tcgen05 kernels (groups of about 66 rows take the 128-row layout,
+    # about 150 rows a full tile and a 22-row one, 21-25 rows the
+    # operand-swapped tile).  x, A, B in {-1,0,1},
     # y in [-8,8]: |buf| <= D and |y| <= 8 + 16 D stay exact (fp16: <= 1032
     # < 2048; bf16: <= 136 < 256), through the hi + lo split as well, so the
     # GPU equals the oracle bit for bit.
