@@ -356,8 +356,12 @@ def step_calls(p, d, what="step"):
         return
     if what in ("step", "fused"):
         # the public one-call per-token path: one fused launch when the shape
-        # fits, else group + shrink + expand; plain stream order
-        ops.bgmv(d.x, d.A, d.B, d.idx, d.y, d.buf, d.meta, p.scale, y_col_off=p.col_off)
+        # fits (plain stream order), else group + shrink + expand with
+        # LORA_FLAG_PDL_EARLY, whose promise holds here: the launch before a
+        # step is the previous step's expand, which writes y only (in a model
+        # it is the base GEMM, which writes y as well)
+        ops.bgmv(d.x, d.A, d.B, d.idx, d.y, d.buf, d.meta, p.scale, y_col_off=p.col_off,
+                 pdl_early=not fused(p))
         return
     if what == "group":
         ops.group(d.idx, p.S, d.meta)
@@ -981,7 +985,9 @@ def run_ours(args):
         "config": {"workload": config_label(p),
                    "step": ("segment shrink + expand" if p.segmented else
                             "one lora_bgmv call: group-by-slot + shrink + expand, "
-                            + ("one fused launch" if ff else f"{launches} launches")),
+                            + ("one fused launch" if ff else
+                               f"{launches} launches, LORA_FLAG_PDL_EARLY (the launch before "
+                               "a step writes none of A, B, idx)")),
                    "l2": l2_desc,
                    "graph": "K steps replayed from CUDA graphs of up to 64 steps, "
                             "the same graphs replayed once untimed first",

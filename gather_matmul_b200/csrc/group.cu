@@ -164,7 +164,7 @@ constexpr int kCntPitch = kGroupWarps + 1;
 //      indices is still in registers); CTA 0 writes the slot offsets and
 //      header, the work items are shared out by key.
 __global__ void __launch_bounds__(kGroupThreads, 1)
-group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ meta) {
+group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ meta, int early) {
   extern __shared__ int smem[];
   const int K = S + 1;
   int* cnt = smem;                          // [key][kCntPitch]
@@ -174,7 +174,11 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
   int* ni = pre + K;                        // items per key, then item offsets
   int* scratch = ni + K;                    // 128 ints of scan scratch, 2 totals, a flag
 
-  ptx::grid_dep_wait();               // the previous kernel's writes (idx, meta) are visible
+  // the previous kernel's writes (idx, meta) are visible after this wait; with
+  // `early` the indices are known not to be among them, and the wait comes
+  // after counting, before the first write to the workspace (a kernel before
+  // this one may still read the grouping held there)
+  if (!early) ptx::grid_dep_wait();
   ptx::grid_dep_launch_dependents();
   MetaLayout L(T, S);
   MetaHeader* hdr = reinterpret_cast<MetaHeader*>(meta);
@@ -222,6 +226,7 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
+  if (early) ptx::grid_dep_wait();
   if (lane == 0 && bad) atomicAdd(&hdr->bad_index, bad);
   __syncthreads();
 
@@ -412,7 +417,8 @@ size_t group_smem_bytes(int S) {
   return sizeof(int) * ((size_t)(kCntPitch + 4) * (S + 1) + 131);
 }
 
-cudaError_t launch_group(int T, int S, const int32_t* idx, void* meta, cudaStream_t st) {
+cudaError_t launch_group(int T, int S, const int32_t* idx, void* meta, cudaStream_t st,
+                         int early) {
   size_t smem = group_smem_bytes(S);
   cudaError_t e = cudaFuncSetAttribute(group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
@@ -425,7 +431,8 @@ cudaError_t launch_group(int T, int S, const int32_t* idx, void* meta, cudaStrea
   cudaLaunchAttribute attr[1] = {pdl_attribute()};
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return counted_launch(cudaLaunchKernelEx(&cfg, group_kernel, T, S, idx, static_cast<char*>(meta)));
+  return counted_launch(
+      cudaLaunchKernelEx(&cfg, group_kernel, T, S, idx, static_cast<char*>(meta), early));
 }
 
 cudaError_t launch_segment_items(int T, int S, int n_seg, const int32_t* seg_starts,

@@ -93,7 +93,11 @@ cudaError_t launch_bgmv_fused(lora_dtype dt, const FusedArgs& a, cudaStream_t st
 
 size_t group_smem_bytes(int S);
 cudaError_t launch_set_ranks(int S, const int32_t* ranks, void* meta, cudaStream_t st);
-cudaError_t launch_group(int T, int S, const int32_t* idx, void* meta, cudaStream_t st);
+// early: idx is not written by the previous launch on the stream, so the
+// grouping reads and counts it before waiting for that launch (programmatic
+// dependent launch) and waits only before writing the workspace
+cudaError_t launch_group(int T, int S, const int32_t* idx, void* meta, cudaStream_t st,
+                         int early = 0);
 cudaError_t launch_segment_items(int T, int S, int n_seg, const int32_t* seg_starts,
                                  const int32_t* seg_adapter, void* meta, cudaStream_t st);
 

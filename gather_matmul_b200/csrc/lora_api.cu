@@ -110,15 +110,21 @@ lora_status lora_workspace_reset(void* meta, size_t meta_bytes, lora_stream_t st
   return from_cuda(cudaMemsetAsync(meta, 0, meta_bytes, (cudaStream_t)stream));
 }
 
-lora_status lora_group(int T, int S, const int32_t* idx, void* meta, size_t meta_bytes,
-                       lora_stream_t stream) {
+// early: idx is not written by the previous launch on the stream
+static lora_status group_impl(int T, int S, const int32_t* idx, void* meta, size_t meta_bytes,
+                              lora_stream_t stream, int early) {
   if (T < 0 || S < 0) return LORA_ERR_INVALID_ARG;
   if (T > LORA_MAX_TOKENS || S < 1 || S > LORA_MAX_SLOTS) return LORA_ERR_UNSUPPORTED;
   if (meta == nullptr || (T > 0 && idx == nullptr)) return LORA_ERR_INVALID_ARG;
   if (!aligned16(meta)) return LORA_ERR_MISALIGNED;
   if (meta_bytes < lora_workspace_bytes(T, S)) return LORA_ERR_INVALID_ARG;
   cudaGetLastError();
-  return from_cuda(launch_group(T, S, idx, meta, (cudaStream_t)stream));
+  return from_cuda(launch_group(T, S, idx, meta, (cudaStream_t)stream, early));
+}
+
+lora_status lora_group(int T, int S, const int32_t* idx, void* meta, size_t meta_bytes,
+                       lora_stream_t stream) {
+  return group_impl(T, S, idx, meta, meta_bytes, stream, 0);
 }
 
 lora_status lora_set_slot_ranks(int S, const int32_t* ranks, void* meta, size_t meta_bytes,
@@ -341,7 +347,7 @@ lora_status lora_bgmv(lora_dtype dtype, int T, int D, int r, int S, int n_slices
   cudaError_t e = launch_bgmv_fused(dtype, f, st);
   if (e != cudaErrorNotSupported) return from_cuda(e);
   cudaGetLastError();
-  s = lora_group(T, S, idx, meta, meta_bytes, stream);
+  s = group_impl(T, S, idx, meta, meta_bytes, stream, (flags & LORA_FLAG_PDL_EARLY) ? 1 : 0);
   if (s != LORA_OK) return s;
   // a successful lora_shrink is exactly one launch on `stream`: the expand's
   // predecessor

@@ -238,8 +238,10 @@ LORA_API lora_status lora_expand(lora_dtype dtype, int T, int r, int S, int n_sl
  *   flags         LORA_FLAG_PDL_EARLY: A, B and idx are not written by the
  *                 kernel launched just before this call on `stream`, so the
  *                 call may read them before that kernel has finished
- *                 (programmatic dependent launch); x and y are always read
- *                 after it.  0: nothing is read before it finishes.
+ *                 (programmatic dependent launch): the one-launch kernel reads
+ *                 A and idx early, the grouping of the three-launch path reads
+ *                 and counts idx early; x, y and the workspace are always read
+ *                 or written after it.  0: nothing is read before it finishes.
  *   meta          workspace as for lora_group (its error counters are used;
  *                 the three-launch path also keeps the grouping there).
  *   Other arguments as for lora_shrink / lora_expand.

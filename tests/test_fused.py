@@ -148,3 +148,29 @@ def test_fused_no_active_does_nothing():
     run_bgmv(d)     # the kernel itself: zero intermediate rows, y untouched
     torch.cuda.synchronize()
     assert torch.all(d.buf == 0) and torch.equal(d.y, y0)
+
+
+def test_back_to_back_calls_share_a_workspace_with_early_grouping():
+    # Two three-launch lora_bgmv calls (grouping, shrink, expand) on ONE
+    # workspace, different batches, LORA_FLAG_PDL_EARLY: the second call's
+    # grouping reads and counts its indices while the first call's expand may
+    # still be reading the grouping held in the workspace; it must write the
+    # workspace only after that expand has finished.  Both results against the
+    # oracle.
+    p1 = W.config(5)[0]
+    p2 = W.make_problem(p1.name, p1.dtype, p1.T, p1.D, p1.r, p1.S, p1.d_out, p1.scale,
+                        seed=77, idx_kind="uniform_neg")
+    assert ops.bgmv_launches(W.TORCH_DTYPE[p1.dtype], p1.T, p1.D, p1.r, p1.S, p1.d_out) == 3
+    d1, d2 = Dev(p1), Dev(p2)
+    d2.meta = d1.meta
+    for _ in range(2):             # the second round also follows a call on the same stream
+        d1.y.copy_(Dev(p1).y)
+        d2.y.copy_(Dev(p2).y)
+        run_bgmv(d1, pdl_early=True)
+        run_bgmv(d2, pdl_early=True)
+    torch.cuda.synchronize()
+    for p, d in ((p1, d1), (p2, d2)):
+        buf_ref, cabs = oracle_shrink(p)
+        assert_buf_close(d.buf, buf_ref, cabs)
+        assert_y_close(p, d.y, oracle_expand(p, buf_ref), "y (end to end)")
+    assert ops.check_errors(d1.meta) == _lib.LORA_OK
