@@ -349,9 +349,11 @@ def step_calls(p, d, what="step"):
     shared = p.shared_A and p.n_slices > 1
     buf = d.buf[0] if shared else d.buf
     if p.segmented:
-        if what in ("step", "shrink"):
+        if what == "step":       # the public one-call segment path: shrink + expand
+            ops.sgmv(d.x, d.A, d.B, d.ss, d.sa, d.y, d.buf, d.meta, p.scale, y_col_off=p.col_off)
+        if what == "shrink":
             ops.shrink_segment(d.x, d.A, d.ss, d.sa, d.buf, d.meta)
-        if what in ("step", "expand"):
+        if what == "expand":
             ops.expand_segment(buf, d.B, d.ss, d.sa, d.y, d.meta, p.scale, y_col_off=p.col_off)
         return
     if what in ("step", "fused"):
@@ -983,7 +985,7 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": W.DTYPE_NAME[p.dtype], "data": "synthetic (seeded normal inputs, random adapters)",
         "config": {"workload": config_label(p),
-                   "step": ("segment shrink + expand" if p.segmented else
+                   "step": ("one lora_sgmv call: segment shrink + expand, 2 launches" if p.segmented else
                             "one lora_bgmv call: group-by-slot + shrink + expand, "
                             + ("one fused launch" if ff else
                                f"{launches} launches, LORA_FLAG_PDL_EARLY (the launch before "

@@ -40,6 +40,8 @@ SIGNATURES = {
     "lora_bgmv": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _i32, _vp, _vp, _f32,
                          _vp, _i64, _vp, _vp, _vp, _i32, ctypes.c_uint, _vp, _sz, _vp]),
     "lora_bgmv_launches": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp]),
+    "lora_sgmv": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _i32, _vp, _vp, _f32,
+                         _vp, _i64, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _sz, _vp]),
     "lora_check_errors": (_i32, [_vp, _sz, _vp]),
     "lora_shrink_noalloc": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp,
                                    _vp, _i32, _vp]),

@@ -270,13 +270,16 @@ lora_status lora_shrink_segment(lora_dtype dtype, int T, int D, int r, int S, in
   return from_cuda(e);
 }
 
-lora_status lora_expand_segment(lora_dtype dtype, int T, int r, int S, int n_slices,
-                                const float* buf, int64_t buf_slice_stride,
-                                const void* const* B, const int32_t* D_out,
-                                const int32_t* seg_starts, const int32_t* seg_adapter,
-                                int n_seg, float scale, void* y, int64_t ldy,
-                                const int64_t* y_col_off, int has_active, void* meta,
-                                size_t meta_bytes, lora_stream_t stream) {
+// after_shrink: the previous launch on the stream is lora_shrink_segment's
+// kernel for this batch (lora_sgmv)
+static lora_status expand_segment_impl(lora_dtype dtype, int T, int r, int S, int n_slices,
+                                       const float* buf, int64_t buf_slice_stride,
+                                       const void* const* B, const int32_t* D_out,
+                                       const int32_t* seg_starts, const int32_t* seg_adapter,
+                                       int n_seg, float scale, void* y, int64_t ldy,
+                                       const int64_t* y_col_off, int has_active, void* meta,
+                                       size_t meta_bytes, lora_stream_t stream,
+                                       int after_shrink) {
   lora_status s = check_expand(dtype, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, y,
                                ldy, y_col_off, meta, meta_bytes);
   if (s != LORA_OK) return s;
@@ -286,6 +289,7 @@ lora_status lora_expand_segment(lora_dtype dtype, int T, int r, int S, int n_sli
   ExpandArgs a = {};
   fill_expand(a, T, r, S, n_slices, buf, buf_slice_stride, B, D_out, nullptr, scale, y, ldy,
               y_col_off, meta);
+  a.after_shrink = after_shrink;
   SegArgs sg = {seg_starts, seg_adapter, n_seg};
   cudaStream_t st = (cudaStream_t)stream;
   cudaGetLastError();
@@ -296,6 +300,47 @@ lora_status lora_expand_segment(lora_dtype dtype, int T, int r, int S, int n_sli
     if (e == cudaSuccess) e = launch_expand_items(dtype, a, max_items_segments(T, n_seg), st);
   }
   return from_cuda(e);
+}
+
+lora_status lora_expand_segment(lora_dtype dtype, int T, int r, int S, int n_slices,
+                                const float* buf, int64_t buf_slice_stride,
+                                const void* const* B, const int32_t* D_out,
+                                const int32_t* seg_starts, const int32_t* seg_adapter,
+                                int n_seg, float scale, void* y, int64_t ldy,
+                                const int64_t* y_col_off, int has_active, void* meta,
+                                size_t meta_bytes, lora_stream_t stream) {
+  return expand_segment_impl(dtype, T, r, S, n_slices, buf, buf_slice_stride, B, D_out,
+                             seg_starts, seg_adapter, n_seg, scale, y, ldy, y_col_off, has_active,
+                             meta, meta_bytes, stream, 0);
+}
+
+lora_status lora_sgmv(lora_dtype dtype, int T, int D, int r, int S, int n_slices, const void* x,
+                      int64_t ldx, const void* const* A, int shared_A, const void* const* B,
+                      const int32_t* D_out, float scale, void* y, int64_t ldy,
+                      const int64_t* y_col_off, float* buf, const int32_t* seg_starts,
+                      const int32_t* seg_adapter, int n_seg, int has_active, void* meta,
+                      size_t meta_bytes, lora_stream_t stream) {
+  const int n_a = shared_A ? 1 : n_slices;
+  if (n_slices < 1 || n_slices > LORA_MAX_SLICES) return LORA_ERR_UNSUPPORTED;
+  if (A == nullptr && T > 0) return LORA_ERR_INVALID_ARG;
+  const int64_t stride = shared_A ? 0 : (int64_t)T * r;
+  lora_status s = check_shrink(dtype, T, D, r, S, n_a, x, ldx, A, buf, meta, meta_bytes);
+  if (s != LORA_OK) return s;
+  s = check_expand(dtype, T, r, S, n_slices, buf, stride, B, D_out, y, ldy, y_col_off, meta,
+                   meta_bytes);
+  if (s != LORA_OK) return s;
+  s = check_segments(T, n_seg, seg_starts, seg_adapter);
+  if (s != LORA_OK) return s;
+  if (!has_active || T == 0) return LORA_OK;
+  // the segment shrink launches only kernels that write buf, the workspace's
+  // work list and its error counters, none of which the tensor-core expand
+  // reads before its wait
+  s = lora_shrink_segment(dtype, T, D, r, S, n_a, x, ldx, A, seg_starts, seg_adapter, n_seg, buf,
+                          1, meta, meta_bytes, stream);
+  if (s != LORA_OK) return s;
+  return expand_segment_impl(dtype, T, r, S, n_slices, buf, stride, B, D_out, seg_starts,
+                             seg_adapter, n_seg, scale, y, ldy, y_col_off, 1, meta, meta_bytes,
+                             stream, 1);
 }
 
 static void fill_fused(FusedArgs& f, int T, int D, int r, int S, int n_slices, const void* x,

@@ -239,6 +239,27 @@ def expand_segment(buf, B, seg_starts, seg_adapter, y, meta, scale=1.0, y_col_of
     return y
 
 
+def sgmv(x: torch.Tensor, A: Sequence[torch.Tensor], B: Sequence[torch.Tensor],
+         seg_starts: torch.Tensor, seg_adapter: torch.Tensor, y: torch.Tensor, buf: torch.Tensor,
+         meta: torch.Tensor, scale: float = 1.0, y_col_off=None, has_active: bool = True,
+         stream=None):
+    """shrink_segment() + expand_segment() of one prefill batch in one call
+    (the expand starts while the shrink finishes).  A: one stack per slice of
+    B, or a single stack shared by every slice; buf: float32 [len(A), T, r]."""
+    T, D, ldx = _xinfo(x)
+    S, r, _ = A[0].shape
+    n = len(B)
+    shared = len(A) == 1 and n > 1
+    if not shared and len(A) != n:
+        raise ValueError("A must hold one stack per slice, or one shared stack")
+    _, ldy, _, _, _, d_out, off, _ = _expand_common(buf, B, y, y_col_off, None)
+    _check("lora_sgmv", _lib.load().lora_sgmv(
+        _dtype(x), T, D, r, S, n, _ptr(x), ldx, _ptrs(A), int(shared), _ptrs(B), d_out,
+        ctypes.c_float(scale), _ptr(y), ldy, off, _ptr(buf), _ptr(seg_starts), _ptr(seg_adapter),
+        seg_adapter.numel(), int(bool(has_active)), _ptr(meta), meta.numel(), _stream(stream)))
+    return y
+
+
 def shrink_noalloc(x: torch.Tensor, A: Sequence[torch.Tensor], idx: torch.Tensor,
                    buf: torch.Tensor, has_active: bool = True, stream=None) -> torch.Tensor:
     """group() + shrink() in one call that needs no workspace: the library keeps

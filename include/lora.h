@@ -292,6 +292,27 @@ LORA_API lora_status lora_expand_segment(lora_dtype dtype, int T, int r, int S, 
                                 size_t meta_bytes, lora_stream_t stream);
 
 /*
+ * SGMV shrink + expand of one prefill batch in one call ("Add multi-LoRA
+ * support", Limitations list: SGMV is the prefill kernel): lora_shrink_segment
+ * into buf, then lora_expand_segment from it, with A either one stack per
+ * slice or (shared_A != 0) one stack whose intermediate every slice expands
+ * (buf then holds one slice).  The result equals the two calls; inside this
+ * call the expand's previous launch is known to be this library's shrink,
+ * which writes only buf, so the tensor-core expand sets up its schedule and
+ * issues its first B and y tiles while the shrink finishes and waits for it
+ * only before reading buf (programmatic dependent launch).
+ *   Arguments as for lora_shrink_segment / lora_expand_segment and lora_bgmv
+ *   (buf: device fp32 [n_A, T, r], n_A = shared_A ? 1 : n_slices).
+ */
+LORA_API lora_status lora_sgmv(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
+                               const void* x, int64_t ldx, const void* const* A, int shared_A,
+                               const void* const* B, const int32_t* D_out, float scale, void* y,
+                               int64_t ldy, const int64_t* y_col_off, float* buf,
+                               const int32_t* seg_starts, const int32_t* seg_adapter, int n_seg,
+                               int has_active, void* meta, size_t meta_bytes,
+                               lora_stream_t stream);
+
+/*
  * Synchronise `stream`, read and clear the workspace's error counter.
  * Returns LORA_ERR_BAD_INDEX if any call since the last check saw an index
  * outside [-1, S) or malformed segments, LORA_ERR_CUDA if the stream reports

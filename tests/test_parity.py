@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 import torch
 
+from gather_matmul_b200 import _lib, ops
 from gather_matmul_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -176,3 +177,48 @@ def test_grouped_random_batches(seed):
                        D=int(rng.choice([128, 776, 2048])), r=r, S=S, d_out=d_out, scale=1.25,
                        seed=400 + seed, idx_kind=kind, frac_neg=0.2)
     _run_and_check(p)
+
+
+def _sgmv_case(name):
+    if name == "prefill-full-size":
+        return W.config(4)[0]
+    if name == "mixed":
+        rng = np.random.default_rng(21)
+        lens = rng.choice([0, 1, 37, 64, 65, 128, 200, 513], size=30)
+        ss = np.concatenate([[0], np.cumsum(lens)])
+        sa = rng.integers(-1, 6, size=30)
+        return W.make_problem("sgmv_mixed", W.BF16, T=int(ss[-1]), D=1024, r=32, S=6,
+                              d_out=[512, 136], scale=0.5, seed=21, segments=(ss, sa))
+    if name == "long-list":                     # > 2048 segments: CUDA-core item kernels
+        ss, sa = _many_segments(2050, 2, 5, 4)
+        return W.make_problem("sgmv_long", W.F16, T=int(ss[-1]), D=256, r=32, S=5,
+                              d_out=[256], scale=1.5, seed=22, segments=(ss, sa))
+    ss, sa = np.array([0, 100, 300, 301, 700]), np.array([2, -1, 0, 3])
+    return W.make_problem("sgmv_shared", W.F16, T=700, D=512, r=64, S=4,
+                          d_out=[256, 128, 128], scale=2.0, seed=23, segments=(ss, sa),
+                          shared_A=True)
+
+
+@pytest.mark.parametrize("name", ["prefill-full-size", "mixed", "long-list", "shared-A"])
+def test_sgmv_one_call(name):
+    """lora_sgmv (segment shrink + expand in one call, the expand started
+    while the shrink finishes) against the oracle."""
+    p = _sgmv_case(name)
+    d = Dev(p)
+    buf_ref, cabs = oracle_shrink(p)
+    ops.sgmv(d.x, d.A, d.B, d.ss, d.sa, d.y, d.buf, d.meta, p.scale, y_col_off=p.col_off)
+    torch.cuda.synchronize()
+    assert_buf_close(d.buf, buf_ref, cabs)
+    assert_y_close(p, d.y, oracle_expand(p, buf_ref), "y (end to end)")
+    assert ops.check_errors(d.meta) == _lib.LORA_OK
+
+
+def test_sgmv_one_call_idle_writes_nothing():
+    p = _sgmv_case("mixed")
+    d = Dev(p)
+    y0 = d.y.clone()
+    ops.sgmv(d.x, d.A, d.B, d.ss, d.sa, d.y, d.buf, d.meta, p.scale, y_col_off=p.col_off,
+             has_active=False)
+    torch.cuda.synchronize()
+    assert torch.equal(d.y, y0)
+    assert torch.isnan(d.buf).all()
