@@ -58,7 +58,7 @@ struct TileInfo {
 // separately).  Warp-cooperative; every lane returns the same answer.
 __device__ bool find_tile(int tile, const int32_t* __restrict__ ss,
                           const int32_t* __restrict__ sa, int n_seg, int T, TileInfo& ti,
-                          int implicit_slots) {
+                          int implicit_slots, int trows = kTM) {
   const int lane = threadIdx.x & 31;
   int base = 0;
   for (int s0 = 0; s0 < n_seg; s0 += 32) {
@@ -68,7 +68,7 @@ __device__ bool find_tile(int tile, const int32_t* __restrict__ ss,
       a = min(max(ss[s], 0), T);
       b = max(a, min(max(ss[s + 1], 0), T));
     }
-    const int nt = (b - a + kTM - 1) / kTM;
+    const int nt = (b - a + trows - 1) / trows;
     int inc = nt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -83,8 +83,8 @@ __device__ bool find_tile(int tile, const int32_t* __restrict__ ss,
       const int sb_l = __shfl_sync(0xffffffffu, b, l);
       const int excl = __shfl_sync(0xffffffffu, inc - nt, l);
       ti.seg = s0 + l;
-      ti.m0 = sa_l + (tile - base - excl) * kTM;
-      ti.valid = min(kTM, sb_l - ti.m0);
+      ti.m0 = sa_l + (tile - base - excl) * trows;
+      ti.valid = min(trows, sb_l - ti.m0);
       // per-token grouping: segment g is slot g, the last one holds the tokens
       // without an adapter
       ti.adapter = implicit_slots ? (s0 + l < implicit_slots ? s0 + l : -1) : sa[s0 + l];
@@ -130,6 +130,7 @@ struct ShrinkTCParams {
   const int32_t* idx;                    // per-token indices checked against the grouping
   int implicit_slots;                    // > 0: segment g is slot g (per-token grouping)
   int T, D, S, n_slices, KS;
+  int trows;                             // rows per tile (<= kTM, the MMA's M)
   int* bad_index;
   int* bad_meta;
   const char* meta;                      // workspace: per-slot ranks
@@ -162,6 +163,14 @@ static_assert(2 * (ShrinkSmem<16>::kTotal + 1024) <= 228 * 1024 &&
 // warps 0-3: loads (one per SM sub-partition, so small gathers issue four-wide),
 // then the epilogue on TMEM lane quadrant = warp; warp 4: MMA issue.
 constexpr int kShrThreads = 160;
+// Rows per shrink tile: 96 for a per-token grouping over 64 or more slots,
+// else 128 (the MMA's M either way; a 96-row tile leaves a quarter of the
+// accumulator unused).  Over many slots a few popular slots' full tiles are
+// the kernel's long poles; cutting them at 96 rows shortens them while the
+// grid still fits one wave: large mixed batch 34.8 us against 39.2 (88 rows:
+// the same, 80 or 64: 50 us, as the extra tiles no longer fit one wave).
+// Batches over few slots keep 128 (96 adds empty CTAs: decode +0.3 us).
+constexpr int kShrManySlots = 64, kShrRowsManySlots = 96;
 
 template <typename E, int R>
 __global__ void __launch_bounds__(kShrThreads, 2)
@@ -199,7 +208,7 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
     const int has_ranks = hdr->has_ranks;
     TileInfo ti;
     const bool found = find_tile(blockIdx.x / KS, P.seg_starts, P.seg_adapter, P.n_seg, P.T, ti,
-                                 P.implicit_slots);
+                                 P.implicit_slots, P.trows);
     const bool meta_ok = hT == P.T && hS == P.S;
     if (!meta_ok && lane == 0 && blockIdx.x == 0 && slice == 0) atomicAdd(P.bad_meta, 1);
     if (lane == 0) {
@@ -1170,7 +1179,8 @@ cudaError_t shrink_tc_launch(const ShrinkArgs& a, const SegArgs& sg, lora_dtype 
   P.n_slices = a.n_slices;
   P.bad_index = const_cast<int*>(&hdr->bad_index);
   P.bad_meta = const_cast<int*>(&hdr->bad_meta);
-  const int max_tiles = (a.T + kTM - 1) / kTM + sg.n_seg;
+  P.trows = implicit_slots >= kShrManySlots ? kShrRowsManySlots : kTM;
+  const int max_tiles = (a.T + P.trows - 1) / P.trows + sg.n_seg;
   const int nkb_all = (a.D + kBK - 1) / kBK;
   // split K across a cluster when there are too few tiles for about 1.5 CTAs
   // per SM, each rank keeping at least 8 K blocks: up to 16 ranks (a

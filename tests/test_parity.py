@@ -222,3 +222,21 @@ def test_sgmv_one_call_idle_writes_nothing():
     torch.cuda.synchronize()
     assert torch.equal(d.y, y0)
     assert torch.isnan(d.buf).all()
+
+
+@pytest.mark.parametrize("seed", list(range(4)))
+def test_grouped_many_slots(seed):
+    """Per-token batches over 64 or more slots: the shrink cuts tiles at 96
+    rows (a slot's tokens then span full 96-row tiles and a short last one,
+    of every length), with skewed, uniform and one-hot popularity and tokens
+    without an adapter."""
+    rng = np.random.default_rng(500 + seed)
+    S = int(rng.integers(64, 200))
+    T = int(16 * S + rng.integers(0, 900))
+    kind = ["zipf", "uniform_neg", "frac_neg", "single"][seed]
+    r = [32, 16, 64, 32][seed]
+    d_out = [[512], [136, 64], [256], [392, 8]][seed]
+    p = W.make_problem("many_slots", W.BF16 if seed % 2 else W.F16, T=T,
+                       D=int(rng.choice([512, 1032, 4096])), r=r, S=S, d_out=d_out, scale=0.75,
+                       seed=600 + seed, idx_kind=kind, frac_neg=0.15)
+    _run_and_check(p)
