@@ -1051,10 +1051,19 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
               ptx::fence_proxy_async_smem();
             }
           } else {
-            // swapped: thread = output column 32q + lane, all groups of 8 tokens
+            // swapped: thread = output column 32q + lane, all groups of 8 tokens.
+            // Each group's result goes back into the stage, then the warp
+            // stores its own 32 columns of those 8 rows as 16-byte pieces
+            // (lane -> row 8g + lane / 4, piece lane % 4): no barrier across
+            // the group's warps, and a group's stores overlap the next
+            // group's tensor-memory load.
             const int col = q * 32 + lane;
             const int hc = col >> 6, cc = col & 63;
             char* cbase = ys + hc * L::kYHalf + (cc & 7) * 2;
+            const int rq = lane >> 2, pc = (q & 1) * 4 + (lane & 3);
+            const char* hbase = ys + (q >> 1) * L::kYHalf;
+            E* ydst = ycol + n0 + q * 32 + 8 * (lane & 3);
+            const bool pc_ok = q * 32 + 8 * (lane & 3) < nn;
             const int ng = (rn.valid + 7) / 8;
             for (int g = 0; g < ng; ++g) {
               uint32_t r[8];
@@ -1077,30 +1086,18 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
                 if (8 * g + v < rn.valid)
                   *py[v] = Elem<E>::from_f32(
                       fmaf(P.scale, __uint_as_float(r[v]) * iv[v], Elem<E>::to_f32(yv[v])));
+              __syncwarp();
+              const int row = 8 * g + rq;
+              if (row < rn.valid && pc_ok) {
+                const int tk = toks[row];
+                if (tk >= 0)
+                  *reinterpret_cast<uint4*>(ydst + (size_t)tk * P.ldy) =
+                      *reinterpret_cast<const uint4*>(hbase + row * 128 + ((pc ^ (row & 7)) << 4));
+              }
             }
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive_cnt(&accempty[a], 2);   // four warps count as eight
-            asm volatile("bar.sync %0, 128;" ::"r"(1 + h) : "memory");   // the group's columns done
-            // rows 0 .. valid-1, 16 chunks each: e -> (row e / 16, chunk e % 16);
-            // at most 64 rows: eight pieces per thread, all read before any store
-            const int gl = q * 32 + lane;
-            uint4 v[8];
-#pragma unroll
-            for (int it = 0; it < 8; ++it) {
-              const int e = gl + 128 * it;
-              const int mr = min(e >> 4, kSwapMax - 1), hh = (e >> 3) & 1, ch = e & 7;
-              v[it] = *reinterpret_cast<const uint4*>(ys + hh * L::kYHalf + mr * 128 +
-                                                      ((ch ^ (mr & 7)) << 4));
-            }
-#pragma unroll
-            for (int it = 0; it < 8; ++it) {
-              const int e = gl + 128 * it;
-              const int mr = e >> 4, hh = (e >> 3) & 1, ch = e & 7;
-              if (mr < rn.valid && 64 * hh + 8 * ch < nn && toks[mr] >= 0)
-                *reinterpret_cast<uint4*>(ycol + (size_t)toks[mr] * P.ldy + n0 + 64 * hh + 8 * ch) =
-                    v[it];
-            }
             ptx::fence_proxy_async_smem();
           }
           __syncwarp();
