@@ -1052,53 +1052,52 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
             }
           } else {
             // swapped: thread = output column 32q + lane, all groups of 8 tokens.
-            // Each group's result goes back into the stage, then the warp
-            // stores its own 32 columns of those 8 rows as 16-byte pieces
-            // (lane -> row 8g + lane / 4, piece lane % 4): no barrier across
-            // the group's warps, and a group's stores overlap the next
-            // group's tensor-memory load.
-            const int col = q * 32 + lane;
-            const int hc = col >> 6, cc = col & 63;
-            char* cbase = ys + hc * L::kYHalf + (cc & 7) * 2;
-            const int rq = lane >> 2, pc = (q & 1) * 4 + (lane & 3);
-            const char* hbase = ys + (q >> 1) * L::kYHalf;
-            E* ydst = ycol + n0 + q * 32 + 8 * (lane & 3);
-            const bool pc_ok = q * 32 + 8 * (lane & 3) < nn;
+            // The 8 x 8 blocks of (column, token) values are transposed across
+            // the lanes 8c .. 8c+7 by shuffles, so that lane 8c + i holds token
+            // 8g + i for the columns 32q + 8c .. +7: its y row piece is read
+            // from the stage as 16 bytes and written straight to global memory
+            // (the stage is only read, so no proxy fence before its refill).
+            const int i8 = lane & 7, cb = lane >> 3;
+            const int pc = (q & 1) * 4 + cb;
+            const char* hbase = ys + (q >> 1) * L::kYHalf + ((pc ^ i8) << 4);
+            E* ydst = ycol + n0 + q * 32 + 8 * cb;
+            const bool pc_ok = q * 32 + 8 * cb < nn;
             const int ng = (rn.valid + 7) / 8;
             for (int g = 0; g < ng; ++g) {
               uint32_t r[8];
               ptx::tc_ld8(tacc + 8 * g, r);
-              const float4 i0 = *reinterpret_cast<const float4*>(invs + 8 * g);
-              const float4 i1 = *reinterpret_cast<const float4*>(invs + 8 * g + 4);
-              const float iv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
-              // token t = 8g + v sits in row t, whose swizzle phase is t & 7 = v
-              uint16_t* py[8];
-              uint16_t yv[8];
-#pragma unroll
-              for (int v = 0; v < 8; ++v) {
-                py[v] = reinterpret_cast<uint16_t*>(cbase + (8 * g + v) * 128 +
-                                                    (((cc >> 3) ^ v) << 4));
-                yv[v] = *py[v];
-              }
+              const int row = 8 * g + i8;            // row & 7 == i8: its swizzle phase
+              const uint4 yw = *reinterpret_cast<const uint4*>(hbase + row * 128);
+              const float iv = invs[row];
+              const int tk = toks[row];
               ptx::tc_wait_ld();
 #pragma unroll
-              for (int v = 0; v < 8; ++v)
-                if (8 * g + v < rn.valid)
-                  *py[v] = Elem<E>::from_f32(
-                      fmaf(P.scale, __uint_as_float(r[v]) * iv[v], Elem<E>::to_f32(yv[v])));
-              __syncwarp();
-              const int row = 8 * g + rq;
-              if (row < rn.valid && pc_ok) {
-                const int tk = toks[row];
-                if (tk >= 0)
-                  *reinterpret_cast<uint4*>(ydst + (size_t)tk * P.ldy) =
-                      *reinterpret_cast<const uint4*>(hbase + row * 128 + ((pc ^ (row & 7)) << 4));
+              for (int mk = 4; mk > 0; mk >>= 1) {
+                const bool up = (i8 & mk) != 0;
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                  if (v & mk) continue;
+                  const uint32_t got = __shfl_xor_sync(0xffffffffu, up ? r[v] : r[v | mk], mk);
+                  if (up) r[v] = got;
+                  else r[v | mk] = got;
+                }
+              }
+              if (row < rn.valid && pc_ok && tk >= 0) {
+                float f[8];
+                Elem<E>::to_f32(yw, f);
+                uint32_t o[4];
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                  o[v] = Elem<E>::pack2(
+                      fmaf(P.scale, __uint_as_float(r[2 * v]) * iv, f[2 * v]),
+                      fmaf(P.scale, __uint_as_float(r[2 * v + 1]) * iv, f[2 * v + 1]));
+                *reinterpret_cast<uint4*>(ydst + (size_t)tk * P.ldy) =
+                    make_uint4(o[0], o[1], o[2], o[3]);
               }
             }
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive_cnt(&accempty[a], 2);   // four warps count as eight
-            ptx::fence_proxy_async_smem();
           }
           __syncwarp();
           if (lane == 0 && deferred != s) ptx::mbar_arrive_cnt(&empty[s], swap ? 2u : 1u);
