@@ -176,10 +176,11 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
 
   // the previous kernel's writes (idx, meta) are visible after this wait; with
   // `early` the indices are known not to be among them, and the wait comes
-  // after counting, before the first write to the workspace (a kernel before
-  // this one may still read the grouping held there)
+  // after counting and after the CTAs have exchanged their counts (through
+  // the histogram rows and barrier words that only this kernel uses), before
+  // the first write to the grouping (a kernel before this one may still read
+  // the grouping held there)
   if (!early) ptx::grid_dep_wait();
-  ptx::grid_dep_launch_dependents();
   MetaLayout L(T, S);
   MetaHeader* hdr = reinterpret_cast<MetaHeader*>(meta);
   int* slot_off = reinterpret_cast<int*>(meta + L.off_slot);
@@ -226,7 +227,6 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
-  if (early) ptx::grid_dep_wait();
   if (lane == 0 && bad) atomicAdd(&hdr->bad_index, bad);
   __syncthreads();
 
@@ -279,6 +279,12 @@ group_kernel(int T, int S, const int32_t* __restrict__ idx, char* __restrict__ m
     const int k = e / kGroupWarps, w = e % kGroupWarps;
     cnt[k * kCntPitch + w] += base[k] + pre[k];
   }
+  // The next kernel may start now: this CTA no longer reads the histogram
+  // rows or the barrier words, which a following grouping launch (with
+  // `early`) may use before its own wait.
+  __syncthreads();
+  ptx::grid_dep_launch_dependents();
+  if (early) ptx::grid_dep_wait();
   for (int k = tid; k < K; k += kGroupThreads) {
     if (cta == 0) slot_off[k] = base[k];
     if (k % nb == cta) {

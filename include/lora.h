@@ -240,8 +240,12 @@ LORA_API lora_status lora_expand(lora_dtype dtype, int T, int r, int S, int n_sl
  *                 call may read them before that kernel has finished
  *                 (programmatic dependent launch): the one-launch kernel reads
  *                 A and idx early, the grouping of the three-launch path reads
- *                 and counts idx early; x, y and the workspace are always read
- *                 or written after it.  0: nothing is read before it finishes.
+ *                 and counts idx early and exchanges the counts of its CTAs
+ *                 through its own words of the workspace (words that no other
+ *                 kernel reads), so that kernel must not write the workspace
+ *                 either; x, y and the grouping held in the workspace are
+ *                 always read or written after it.  0: nothing is read before
+ *                 it finishes.
  *   meta          workspace as for lora_group (its error counters are used;
  *                 the three-launch path also keeps the grouping there).
  *   Other arguments as for lora_shrink / lora_expand.

@@ -150,6 +150,30 @@ def test_fused_no_active_does_nothing():
     assert torch.all(d.buf == 0) and torch.equal(d.y, y0)
 
 
+def test_early_grouping_right_after_a_grouping_on_the_same_workspace():
+    # A stand-alone grouping of one batch, then at once a three-launch
+    # lora_bgmv call of another batch with LORA_FLAG_PDL_EARLY on the same
+    # workspace: the second grouping's CTAs exchange their counts through the
+    # workspace before waiting for the first grouping, which must have
+    # finished its own exchange before the second one can start.  Batches of
+    # 4096 tokens use several grouping CTAs.  Result against the oracle.
+    p1 = W.config(5)[0]
+    p2 = W.make_problem(p1.name, p1.dtype, p1.T, p1.D, p1.r, p1.S, p1.d_out, p1.scale,
+                        seed=78, idx_kind="uniform_neg")
+    d1, d2 = Dev(p1), Dev(p2)
+    d2.meta = d1.meta
+    y0 = d2.y.clone()
+    for _ in range(3):
+        d2.y.copy_(y0)
+        ops.group(d1.idx, p1.S, d1.meta)
+        run_bgmv(d2, pdl_early=True)
+    torch.cuda.synchronize()
+    buf_ref, cabs = oracle_shrink(p2)
+    assert_buf_close(d2.buf, buf_ref, cabs)
+    assert_y_close(p2, d2.y, oracle_expand(p2, buf_ref), "y (end to end)")
+    assert ops.check_errors(d1.meta) == _lib.LORA_OK
+
+
 def test_back_to_back_calls_share_a_workspace_with_early_grouping():
     # Two three-launch lora_bgmv calls (grouping, shrink, expand) on ONE
     # workspace, different batches, LORA_FLAG_PDL_EARLY: the second call's
