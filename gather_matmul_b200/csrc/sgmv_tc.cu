@@ -527,21 +527,34 @@ struct ExpandSmem {
   static_assert(kOffChunk % 8 == 0 && kOffSeg % 16 == 0 && kOffBar % 8 == 0, "alignment");
 };
 
-// The time a pair takes on one SM, in quarter nanoseconds, as measured on
-// B200 by a least-squares fit of each CTA's time against its pairs and rows
-// (Zipf, uniform and mixed-size batches at rank 32):
-//   operand-swapped tile (<= kSwapMax rows): 0.58 us + 16.5 ns per valid
-//     row: its epilogue is one round of the pipeline for few rows;
-//   128-row layout (more rows): 1.2 us + 5 ns per valid row, nearly flat:
-//     the whole tile passes through tensor memory and the epilogue;
+// The time a pair takes on one SM, in quarter nanoseconds, from
+// least-squares fits on B200 of each CTA's time against its pairs, their
+// rows and its runs (residual 0.2-1.9 us per CTA):
+//   rank 16 and 32 (a fit over Zipf, uniform, mixed-size, prefill and
+//     fused-slice decode batches):
+//     operand-swapped tile (<= kSwapMax rows): 0.47 us + 16.4 ns per valid
+//     row (its epilogue is one round of the pipeline for few rows);
+//     128-row layout (more rows): 1.56 us + 1.3 ns per valid row, nearly
+//     flat (the whole tile passes through tensor memory and the epilogue);
+//   rank 64: the weights of an earlier fit (0.58 us + 16.5 ns, 1.2 us +
+//     5 ns), which a simulation of the schedule with a rank-64 fit's costs
+//     found as good as any refit (the refit above made the decode gate_up
+//     expand 30.1 -> 31.6 us);
 //   plus about 4.5 ns per rank column of the B tile (its 256 r bytes).
-// Weights in bytes moved rated a full tile at 3.3 small tiles (it costs
-// about 2.8) and a 90-row tile far below a full one (it costs 90 %), which
-// left CTAs of small groups as the long poles.
+// With the earlier weights at rank 32 the CTAs of partial 128-row tiles ran
+// 20 % longer than the mean on the large mixed batch (62 against 52 us);
+// refitted, the large mixed expand went from 66.4 to 64.1 us (a rank-32-only
+// fit: 65.2 us).  Weights in bytes moved had rated a full tile at 3.3 small
+// tiles and a 90-row tile far below a full one, which left CTAs of small
+// groups as the long poles.
 template <int R>
 __device__ __forceinline__ int64_t pair_weight(int valid) {
-  return valid <= kSwapMax ? 1744 + 18 * R + 66 * (int64_t)valid
-                           : 4224 + 18 * R + 20 * (int64_t)valid;
+  if constexpr (R >= 64)
+    return valid <= kSwapMax ? 1744 + 18 * R + 66 * (int64_t)valid
+                             : 4224 + 18 * R + 20 * (int64_t)valid;
+  else
+    return valid <= kSwapMax ? 1320 + 18 * R + 66 * (int64_t)valid
+                             : 5660 + 18 * R + 5 * (int64_t)valid;
 }
 
 // Per n-tile weight of one segment: its full tiles and its partial last tile.
