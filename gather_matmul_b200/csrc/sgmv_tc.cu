@@ -519,7 +519,7 @@ struct ExpandSmem {
   static constexpr size_t kOffChunk = kOffRun + kMaxRuns * sizeof(ExpRun);   // int64 [chunks]
   static constexpr size_t kOffSeg = (kOffChunk + 8 * kMaxSegChunks + 15) & ~size_t(15);   // int4 [kSegCache]
   static constexpr size_t kOffBar = kOffSeg + 16 * kSegCache;
-  static constexpr int kNBar = 2 * kYS + 8;
+  static constexpr int kNBar = 2 * kYS + 10;
   static constexpr size_t kOffMisc = kOffBar + 8 * kNBar;             // tmem, n_runs, next
   static constexpr size_t kTotal = kOffMisc + 64 + 1024;
   static_assert(kOffB % 1024 == 0 && kOffHL % 1024 == 0, "swizzled tiles need 1024-byte alignment");
@@ -687,15 +687,24 @@ __device__ int build_runs(const SegView& sv, const int64_t* chunkW, int64_t Wt,
 }
 
 // warps 0-7: epilogue (TMEM lane quadrant = warp % 4, column half = warp / 4),
-// warps 8-11: loads (one per SM sub-partition), warp 12: MMA issue.
-constexpr int kExpThreads = 416;
-constexpr int kExpLoad0 = 8, kExpMma = 12;
+// warps 8-11: loads (one per SM sub-partition), warp 12: MMA issue, warps
+// 13-: operands (each run's tokens and hi / lo rows, one run ahead): two
+// warps reading two buf rows per lane at once up to rank 32; at rank 64 (a
+// row fills half the registers) three warps reading one row per lane at a
+// time, so the rows of a run of up to 96 tokens are read in one round.
+constexpr int kExpLoad0 = 8, kExpMma = 12, kExpOpnd0 = 13;
+template <int R>
+constexpr int exp_opnd_warps() { return R >= 64 ? 3 : 2; }
+template <int R>
+constexpr int exp_threads() { return 32 * (kExpOpnd0 + exp_opnd_warps<R>()); }
 
 template <typename E, int R>
-__global__ void __launch_bounds__(kExpThreads, 1)
+__global__ void __launch_bounds__(exp_threads<R>(), 1)
 sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   using L = ExpandSmem<R>;
   constexpr int kYS = L::kYS;
+  constexpr int kOW = exp_opnd_warps<R>();             // operand warps
+  constexpr int kRPL = (kTM + 32 * kOW - 1) / (32 * kOW);  // operand rows per lane
   constexpr bool kBF = std::is_same<E, __nv_bfloat16>::value;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // The previous kernel (programmatic dependent launch) is waited for here,
@@ -721,6 +730,7 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   uint64_t* accempty = accfull + 2;      // [2]
   uint64_t* hlfull = accempty + 2;       // [2]
   uint64_t* hlempty = hlfull + 2;        // [2]
+  uint64_t* tokfull = hlempty + 2;       // [2] tokens of operand buffer b written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   int* sNRuns = reinterpret_cast<int*>(tmem_slot + 1);
   int64_t* sRange = reinterpret_cast<int64_t*>(smem + L::kOffMisc + 8);   // lo, hi, Wt, next
@@ -768,7 +778,8 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&accfull[a], 1);
       ptx::mbar_init(&accempty[a], 8);
-      ptx::mbar_init(&hlfull[a], 4);
+      ptx::mbar_init(&hlfull[a], kOW);     // one arrival per operand warp
+      ptx::mbar_init(&tokfull[a], kOW);
       ptx::mbar_init(&hlempty[a], 8);
     }
     ptx::fence_mbar_init();
@@ -800,28 +811,14 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
     const int64_t next_lo = sRange[3];
 
     if (warp >= kExpLoad0 && warp < kExpMma) {
-      // ---------------- loads
+      // ---------------- loads: per pair its B tile and y rows
       const int pw = warp - kExpLoad0;
-      const int lt = pw * 32 + lane;                 // operand row of this thread
       int pl = p, ul = u;
-      bool buf_ready = !P.early;
       for (int ri = 0; ri < n_runs; ++ri, ++ul) {
         const ExpRun rn = runs[ri];
         const int hb = ul & 1;
-        if (ul >= 2) ok &= ptx::mbar_wait_ff(&hlempty[hb], ((ul >> 1) - 1) & 1, sAbort);
-        // this thread's operand row: its token first (the gathers need every
-        // row's token), then the loads of the run's first pairs whose stages
-        // are free without waiting, then the hi / lo rows, so that the buf
-        // reads overlap those loads
-        const int m = lt;
-        // sTok: the row's token; -1 past the tile; -2 - token for a token whose
-        // index disagrees with its group (stale workspace): still a valid row
-        // address for the gathers, but never written back (counted below).
-        // The gathers need only the token, so the index check is made after
-        // they are issued, together with the buf row read.
-        const int tok = m < rn.valid ? (P.perm ? P.perm[rn.m0 + m] : rn.m0 + m) : -1;
-        sTok[hb * kTM + m] = tok;
-        asm volatile("bar.sync 4, 128;" ::: "memory");   // every row's token is known
+        // the run's tokens (written by the operand warps)
+        ok &= ptx::mbar_wait_ff(&tokfull[hb], (ul >> 1) & 1, sAbort);
         const int* toks = sTok + hb * kTM;
         const int Dout = P.D_out[rn.slice];
         const int64_t ycol0 = P.y_col_off[rn.slice];
@@ -830,9 +827,9 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
         int my_ops = 0;
         if (!tiled)
           for (int o = pw; o < 2 * ngroups; o += 4) ++my_ops;
-        auto issue_pair = [&](int j, int pq) {
-          const int s = pq % kYS;
-          if (pq >= kYS) ok &= ptx::mbar_wait_ff(&empty[s], ((pq / kYS) - 1) & 1, sAbort);
+        for (int j = rn.j0; j < rn.j1; ++j, ++pl) {
+          const int s = pl % kYS;
+          if (pl >= kYS) ok &= ptx::mbar_wait_ff(&empty[s], ((pl / kYS) - 1) & 1, sAbort);
           const int n0 = j * kNT;
           char* ys = sY + (size_t)s * L::kYBytes;
           // the B tile holds only the first 16 << kc columns of each row
@@ -866,57 +863,99 @@ sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
                                rr[0], rr[1], rr[2], rr[3], &full[s]);
             }
           }
-        };
-        int j = rn.j0;
-        for (; j < rn.j1 && pl < kYS; ++j, ++pl) issue_pair(j, pl);
-        // hi / lo after an exact power-of-two rescale 2^(7-e) (e = exponent of
-        // the row's max |buf|), and the inverse scale
-        {
-          if (!buf_ready) {
-            ptx::grid_dep_wait();                    // the shrink has written buf
-            buf_ready = true;
-          }
-          const float4* brow = reinterpret_cast<const float4*>(
-              P.buf + (size_t)rn.slice * P.buf_slice_stride + (size_t)(tok < 0 ? 0 : tok) * R);
-          const bool stale = tok >= 0 && P.perm && !grouped_row_ok(P.idx, tok, rn.adapter, P.S);
-          float4 f[R / 4];
-          float mx = 0.f;
+        }
+      }
+    } else if (warp >= kExpOpnd0) {
+      // ---------------- operands: per run its tokens, then the hi / lo rows
+      // of its buf rows, while the loads, MMAs and epilogue of the run before
+      // are under way (double-buffered)
+      const int ow = warp - kExpOpnd0;
+      int ul = u;
+      bool buf_ready = !P.early;
+      for (int ri = 0; ri < n_runs; ++ri, ++ul) {
+        const ExpRun rn = runs[ri];
+        const int hb = ul & 1;
+        if (ul >= 2) ok &= ptx::mbar_wait_ff(&hlempty[hb], ((ul >> 1) - 1) & 1, sAbort);
+        // rows the MMA reads: all 128 in the 128-row layout, the valid rows
+        // rounded up to 16 when the operands are swapped
+        const int nrows = rn.valid <= kSwapMax ? (rn.valid + 15) & ~15 : kTM;
+        // sTok: the row's token; -1 past the tile; -2 - token for a token whose
+        // index disagrees with its group (stale workspace): still a valid row
+        // address for the gathers, but never written back (counted below).
+        // The gathers need only the tokens, so the index check is made after
+        // they are published, together with the buf row read.
+        int tk[kRPL];
 #pragma unroll
-          for (int q = 0; q < R / 4; ++q) {
-            f[q] = (tok >= 0 && 4 * q < (16 << rn.kc)) ? brow[q] : make_float4(0.f, 0.f, 0.f, 0.f);
-            mx = fmaxf(fmaxf(fmaxf(mx, fabsf(f[q].x)), fmaxf(fabsf(f[q].y), fabsf(f[q].z))),
-                       fabsf(f[q].w));
-          }
-          int e = ((__float_as_int(mx) >> 23) & 0xff) - 127;
-          e = (mx > 0.f && e > -100 && e < 100) ? e : 0;
-          const float sc = __int_as_float((127 - e + 7) << 23);
-          char* hiP = sHL + (size_t)(2 * hb) * L::kHBytes;
-          char* loP = hiP + L::kHBytes;
-#pragma unroll
-          for (int c = 0; c < R / 8; ++c) {
-            const float x8[8] = {f[2 * c].x, f[2 * c].y, f[2 * c].z, f[2 * c].w,
-                                 f[2 * c + 1].x, f[2 * c + 1].y, f[2 * c + 1].z, f[2 * c + 1].w};
-            uint16_t h8[8], l8[8];
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              const float xv = x8[v] * sc;
-              h8[v] = Elem<E>::from_f32(xv);
-              l8[v] = Elem<E>::from_f32(xv - Elem<E>::to_f32(h8[v]));
-            }
-            const int off = m * L::kRowBytes + swz<L::kRowBytes>(m, c) * 16;
-            *reinterpret_cast<uint4*>(hiP + off) = *reinterpret_cast<const uint4*>(h8);
-            *reinterpret_cast<uint4*>(loP + off) = *reinterpret_cast<const uint4*>(l8);
-          }
-          sInv[hb * kTM + m] = __int_as_float((127 + e - 7) << 23);
-          if (stale) {
-            if (rn.j0 == 0) atomicAdd(P.bad_meta, 1);
-            sTok[hb * kTM + m] = -2 - tok;   // the gathers read either form as row tok
-          }
-          ptx::fence_proxy_async_smem();   // generic writes -> tensor-core operand reads
+        for (int i = 0; i < kRPL; ++i) {
+          const int m = 32 * (ow + kOW * i) + lane;   // rows past 127 are not read
+          tk[i] = m < rn.valid ? (P.perm ? P.perm[rn.m0 + m] : rn.m0 + m) : -1;
+          if (m < nrows) sTok[hb * kTM + m] = tk[i];
         }
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&hlfull[hb]);   // one arrival per load warp
-        for (; j < rn.j1; ++j, ++pl) issue_pair(j, pl);
+        if (lane == 0) ptx::mbar_arrive(&tokfull[hb]);
+        if (!buf_ready) {
+          ptx::grid_dep_wait();                      // the shrink has written buf
+          buf_ready = true;
+        }
+        // hi / lo after an exact power-of-two rescale 2^(7-e) (e = exponent of
+        // the row's max |buf|), and the inverse scale; rows are read kB at a time
+        constexpr int kB = R <= 32 ? kRPL : 1;
+        char* hiP = sHL + (size_t)(2 * hb) * L::kHBytes;
+        char* loP = hiP + L::kHBytes;
+#pragma unroll
+        for (int i0 = 0; i0 < kRPL; i0 += kB) {
+          float4 f[kB][R / 4];
+#pragma unroll
+          for (int b = 0; b < kB; ++b) {
+            const int m = 32 * (ow + kOW * (i0 + b)) + lane;
+            const int tok = tk[i0 + b];
+            const float4* brow = reinterpret_cast<const float4*>(
+                P.buf + (size_t)rn.slice * P.buf_slice_stride + (size_t)(tok < 0 ? 0 : tok) * R);
+#pragma unroll
+            for (int q = 0; q < R / 4; ++q)
+              f[b][q] = (m < nrows && tok >= 0 && 4 * q < (16 << rn.kc))
+                            ? brow[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int b = 0; b < kB; ++b) {
+            const int m = 32 * (ow + kOW * (i0 + b)) + lane;
+            const int tok = tk[i0 + b];
+            if (m >= nrows) continue;
+            const bool stale = tok >= 0 && P.perm && !grouped_row_ok(P.idx, tok, rn.adapter, P.S);
+            float mx = 0.f;
+#pragma unroll
+            for (int q = 0; q < R / 4; ++q)
+              mx = fmaxf(fmaxf(fmaxf(mx, fabsf(f[b][q].x)), fmaxf(fabsf(f[b][q].y), fabsf(f[b][q].z))),
+                         fabsf(f[b][q].w));
+            int e = ((__float_as_int(mx) >> 23) & 0xff) - 127;
+            e = (mx > 0.f && e > -100 && e < 100) ? e : 0;
+            const float sc = __int_as_float((127 - e + 7) << 23);
+#pragma unroll
+            for (int c = 0; c < R / 8; ++c) {
+              const float x8[8] = {f[b][2 * c].x, f[b][2 * c].y, f[b][2 * c].z, f[b][2 * c].w,
+                                   f[b][2 * c + 1].x, f[b][2 * c + 1].y, f[b][2 * c + 1].z,
+                                   f[b][2 * c + 1].w};
+              uint16_t h8[8], l8[8];
+#pragma unroll
+              for (int v = 0; v < 8; ++v) {
+                const float xv = x8[v] * sc;
+                h8[v] = Elem<E>::from_f32(xv);
+                l8[v] = Elem<E>::from_f32(xv - Elem<E>::to_f32(h8[v]));
+              }
+              const int off = m * L::kRowBytes + swz<L::kRowBytes>(m, c) * 16;
+              *reinterpret_cast<uint4*>(hiP + off) = *reinterpret_cast<const uint4*>(h8);
+              *reinterpret_cast<uint4*>(loP + off) = *reinterpret_cast<const uint4*>(l8);
+            }
+            sInv[hb * kTM + m] = __int_as_float((127 + e - 7) << 23);
+            if (stale) {
+              if (rn.j0 == 0) atomicAdd(P.bad_meta, 1);
+              sTok[hb * kTM + m] = -2 - tok;   // the gathers read either form as row tok
+            }
+          }
+        }
+        ptx::fence_proxy_async_smem();   // generic writes -> tensor-core operand reads
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&hlfull[hb]);   // one arrival per operand warp
       }
     } else if (warp == kExpMma) {
       // ---------------- MMA issue
@@ -1294,7 +1333,7 @@ cudaError_t expand_tc_launch(const ExpandArgs& a, const SegArgs& sg, lora_dtype 
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(kExpThreads, 1, 1);
+  cfg.blockDim = dim3(exp_threads<R>(), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1] = {pdl_attribute()};
