@@ -460,7 +460,7 @@ __device__ __forceinline__ int ceil_pos_nt(int64_t num, int w, int nt) {
 //   load warps   B tile + y tile of each pair into a ring of stages; the
 //                hi / lo operand of each run (double-buffered)
 //   MMA warp     acc = hi . B^T + lo . B^T into one of two TMEM accumulators;
-//                a tile of <= kSwapMax rows swaps the operands (M = 128 output
+//                a tile of <= swap_max<R>() rows swaps the operands (M = 128 output
 //                columns, N = its rows rounded to 16) so the epilogue only
 //                touches the rows that exist
 //   epilogue     y += scale * acc, one rounding; two warps per TMEM lane
@@ -470,10 +470,12 @@ struct ExpRun {
   int kc;        // the adapter's rank rounded up to 16 << kc (per-slot ranks)
 };
 constexpr int kMaxRuns = 64;
-// tiles of at most this many rows swap operands: by the measured pair costs
-// below the two layouts break even near 54 rows (48: large mixed step 114.3 us
-// against 114.8 with 64)
-constexpr int kSwapMax = 48;
+// Tiles of at most swap_max<R>() rows swap operands.  Measured on B200 (one
+// lora_bgmv step): at rank 32, 48 rows (large mixed 97.2 us against 97.5 with
+// 56 and 97.6 with 64); at rank 64, 64 rows (decode qkv / gate_up / down
+// 25.8 / 37.6 / 25.1 us against 26.7 / 39.6 / 26.3 with 48; 56 the same).
+template <int R>
+constexpr int swap_max() { return R >= 64 ? 64 : 48; }
 
 struct ExpandTCParams {
   // B_i as [S*D_out_i rows, r cols], box {16 << c, 128} with a (32 << c)-byte
@@ -532,7 +534,7 @@ struct ExpandSmem {
 // rows and its runs (residual 0.2-1.9 us per CTA):
 //   rank 16 and 32 (a fit over Zipf, uniform, mixed-size, prefill and
 //     fused-slice decode batches):
-//     operand-swapped tile (<= kSwapMax rows): 0.47 us + 16.4 ns per valid
+//     operand-swapped tile (<= swap_max<R>() rows): 0.47 us + 16.4 ns per valid
 //     row (its epilogue is one round of the pipeline for few rows);
 //     128-row layout (more rows): 1.56 us + 1.3 ns per valid row, nearly
 //     flat (the whole tile passes through tensor memory and the epilogue);
@@ -549,6 +551,7 @@ struct ExpandSmem {
 // groups as the long poles.
 template <int R>
 __device__ __forceinline__ int64_t pair_weight(int valid) {
+  constexpr int kSwapMax = swap_max<R>();
   if constexpr (R >= 64)
     return valid <= kSwapMax ? 1744 + 18 * R + 66 * (int64_t)valid
                              : 4224 + 18 * R + 20 * (int64_t)valid;
@@ -703,6 +706,7 @@ __global__ void __launch_bounds__(exp_threads<R>(), 1)
 sgmv_expand_tc_kernel(const __grid_constant__ ExpandTCParams P) {
   using L = ExpandSmem<R>;
   constexpr int kYS = L::kYS;
+  constexpr int kSwapMax = swap_max<R>();
   constexpr int kOW = exp_opnd_warps<R>();             // operand warps
   constexpr int kRPL = (kTM + 32 * kOW - 1) / (32 * kOW);  // operand rows per lane
   constexpr bool kBF = std::is_same<E, __nv_bfloat16>::value;
