@@ -587,18 +587,22 @@ __device__ int64_t seg_chunk_weights(const SegView& sv, int64_t* chunkW, const c
   const int lane = threadIdx.x & 31;
   const int nch = (sv.n_seg + 31) / 32;
   int64_t total = 0;
-  // four chunks per round: all their loads first, then the reductions
+  // four chunks per round: all their segment loads first (ahead of the
+  // shared-memory copies, which the compiler may not move loads across),
+  // then the weights and the reductions
   constexpr int kU = 4;
   for (int c0 = 0; c0 < nch; c0 += kU) {
     int64_t w[kU];
+    int a[kU], b[kU], ad[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) sv.get((c0 + u) * 32 + lane, a[u], b[u], ad[u]);
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      int a, b, ad;
       const int sidx = (c0 + u) * 32 + lane;
-      sv.get(sidx, a, b, ad);
       if (sidx < kSegCache)
-        sv.cache[sidx] = make_int4(a, b, ad, ad >= 0 ? rank_class<R>(meta, sv.S, ad, has_ranks) : 0);
-      w[u] = seg_weight<R>(a, b, ad);
+        sv.cache[sidx] = make_int4(a[u], b[u], ad[u],
+                                   ad[u] >= 0 ? rank_class<R>(meta, sv.S, ad[u], has_ranks) : 0);
+      w[u] = seg_weight<R>(a[u], b[u], ad[u]);
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
