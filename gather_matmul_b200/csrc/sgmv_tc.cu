@@ -343,6 +343,9 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
   }
   ok &= ptx::mbar_wait(accbar, 0);
   ptx::tc_fence_after();
+  // split K: this CTA's MMAs are done, so its stages are drained and may take
+  // the peers' partials; the barrier's latency overlaps the accumulator read
+  if (KS > 1) cluster.barrier_arrive();
 
   // accumulator row m = 32 * warp + lane (warps 0-3), r fp32 columns
   const bool has_row = warp < 4;
@@ -370,8 +373,7 @@ sgmv_shrink_tc_kernel(const __grid_constant__ ShrinkTCParams P) {
     // receive area (the owner's drained stage memory), then each owner adds
     // its KS slots in rank order.
     const int rpr = (valid + KS - 1) / KS;
-    cluster.barrier_arrive();                 // this CTA's MMAs and stages are done...
-    cluster.barrier_wait();                   // ...and so are every peer's
+    cluster.barrier_wait();                   // every peer's MMAs and stages are done
     float* recv = reinterpret_cast<float*>(smem);
     if (has_row && m < valid) {
       float* dst = cluster.map_shared_rank(recv, m / rpr) + (size_t)(kr * rpr + m % rpr) * L::kPitch;
