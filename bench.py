@@ -698,8 +698,9 @@ def configs_block(stream, peak, tf_peak, reps=256):
 def layer_one_grouping(stream, peak, reps):
     """The three fused-slice projections of one decoder layer as a decode
     step runs them: the batch's grouping built once (lora_group) and shared by
-    every projection's shrink and expand (the projections of one batch carry
-    the same indices)."""
+    every projection (the projections of one batch carry the same indices),
+    each projection one lora_bgmv call with LORA_FLAG_GROUPED (shrink, then
+    the chained expand)."""
     from gather_matmul_b200 import ops
     probs = W.config(3)
     sets = [make_sets(p) for p in probs]
@@ -710,8 +711,8 @@ def layer_one_grouping(stream, peak, reps):
         ops.group(d0.idx, probs[0].S, d0.meta)
         for p, ss in zip(probs, sets):
             d = ss[k % n]
-            ops.shrink(d.x, d.A, d0.idx, d.buf, d0.meta)
-            ops.expand(d.buf, d.B, d0.idx, d.y, d0.meta, p.scale, y_col_off=p.col_off)
+            ops.bgmv(d.x, d.A, d.B, d0.idx, d.y, d.buf, d0.meta, p.scale, y_col_off=p.col_off,
+                     grouped=True)
 
     graphs = []
     G = 32

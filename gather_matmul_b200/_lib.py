@@ -22,6 +22,7 @@ LORA_MAX_SLOTS = 1024
 LORA_MAX_TOKENS = 1 << 22
 LORA_NOALLOC_MAX_TOKENS = 8192
 LORA_FLAG_PDL_EARLY = 1
+LORA_FLAG_GROUPED = 2
 
 # Every symbol the header declares, with (restype, argtypes).
 _i32, _i64, _sz, _f32, _vp = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float, ctypes.c_void_p

@@ -392,8 +392,10 @@ lora_status lora_bgmv(lora_dtype dtype, int T, int D, int r, int S, int n_slices
   cudaError_t e = launch_bgmv_fused(dtype, f, st);
   if (e != cudaErrorNotSupported) return from_cuda(e);
   cudaGetLastError();
-  s = group_impl(T, S, idx, meta, meta_bytes, stream, (flags & LORA_FLAG_PDL_EARLY) ? 1 : 0);
-  if (s != LORA_OK) return s;
+  if (!(flags & LORA_FLAG_GROUPED)) {
+    s = group_impl(T, S, idx, meta, meta_bytes, stream, (flags & LORA_FLAG_PDL_EARLY) ? 1 : 0);
+    if (s != LORA_OK) return s;
+  }
   // a successful lora_shrink is exactly one launch on `stream`: the expand's
   // predecessor
   s = lora_shrink(dtype, T, D, r, S, n_a, x, ldx, A, idx, buf, 1, meta, meta_bytes, stream);

@@ -188,12 +188,14 @@ def expand(buf: torch.Tensor, B: Sequence[torch.Tensor], idx: torch.Tensor, y: t
 def bgmv(x: torch.Tensor, A: Sequence[torch.Tensor], B: Sequence[torch.Tensor], idx: torch.Tensor,
          y: torch.Tensor, buf: torch.Tensor, meta: torch.Tensor, scale: float = 1.0,
          y_col_off=None, has_active: Optional[bool] = None, idx_host=None,
-         pdl_early: bool = False, stream=None):
+         pdl_early: bool = False, grouped: bool = False, stream=None):
     """group + shrink + expand of one batch in one call (one launch when the
     shape fits the fused kernel).  A: one stack per slice of B, or a single
     stack shared by every slice; buf: float32 [len(A), T, r] receives the
     intermediate; y is updated in place.  pdl_early=True promises that A, B
-    and idx are not written by the kernel launched just before on the stream."""
+    and idx are not written by the kernel launched just before on the stream;
+    grouped=True that meta already holds this idx's grouping (group(), or an
+    earlier bgmv of the batch): no grouping launch."""
     T, D, ldx = _xinfo(x)
     S, r, _ = A[0].shape
     n = len(B)
@@ -202,7 +204,8 @@ def bgmv(x: torch.Tensor, A: Sequence[torch.Tensor], B: Sequence[torch.Tensor], 
         raise ValueError("A must hold one stack per slice, or one shared stack")
     _, ldy, _, _, _, d_out, off, _ = _expand_common(buf, B, y, y_col_off, None)
     _check_idx(idx, T)
-    flags = _lib.LORA_FLAG_PDL_EARLY if pdl_early else 0
+    flags = (_lib.LORA_FLAG_PDL_EARLY if pdl_early else 0) | \
+        (_lib.LORA_FLAG_GROUPED if grouped else 0)
     _check("lora_bgmv", _lib.load().lora_bgmv(
         _dtype(x), T, D, r, S, n, _ptr(x), ldx, _ptrs(A), int(shared), _ptrs(B), d_out,
         ctypes.c_float(scale), _ptr(y), ldy, off, _ptr(buf), _ptr(idx),

@@ -246,11 +246,20 @@ LORA_API lora_status lora_expand(lora_dtype dtype, int T, int r, int S, int n_sl
  *                 either; x, y and the grouping held in the workspace are
  *                 always read or written after it.  0: nothing is read before
  *                 it finishes.
+ *                 LORA_FLAG_GROUPED: the workspace already holds the grouping
+ *                 of this idx (lora_group, or an earlier lora_bgmv of the same
+ *                 batch, on this stream), as when the projections of one
+ *                 decoder layer share a batch: the three-launch path makes
+ *                 two launches (shrink, expand) and no grouping.  The grouping
+ *                 is checked against idx row by row as in lora_shrink, so a
+ *                 stale one is reported, never used silently.  The one-launch
+ *                 kernel finds its tokens itself and ignores the flag.
  *   meta          workspace as for lora_group (its error counters are used;
  *                 the three-launch path also keeps the grouping there).
  *   Other arguments as for lora_shrink / lora_expand.
  */
 #define LORA_FLAG_PDL_EARLY 1u
+#define LORA_FLAG_GROUPED 2u
 LORA_API lora_status lora_bgmv(lora_dtype dtype, int T, int D, int r, int S, int n_slices,
                                const void* x, int64_t ldx, const void* const* A, int shared_A,
                                const void* const* B, const int32_t* D_out, float scale, void* y,

@@ -169,3 +169,15 @@ def test_has_active_from_host_indices():
     assert ops._active(None, None, 4) == 1          # no host copy: the device decides
     assert ops._active(None, np.array([-1]), 4) == 0
     assert ops._active(False, np.array([0]), 4) == 0   # an explicit flag wins
+
+
+def test_binding_constants_match_the_header():
+    # the flag and size constants of the Python binding are the header's own
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(__file__), "..", "include", "lora.h")).read()
+    defines = {m.group(1): int(m.group(2))
+               for m in re.finditer(r"#define\s+(LORA_FLAG_\w+)\s+(\d+)u", src)}
+    assert defines == {"LORA_FLAG_PDL_EARLY": 1, "LORA_FLAG_GROUPED": 2}
+    for name, value in defines.items():
+        assert getattr(_lib, name) == value, name

@@ -150,6 +150,44 @@ def test_fused_no_active_does_nothing():
     assert torch.all(d.buf == 0) and torch.equal(d.y, y0)
 
 
+def test_grouped_flag_shares_one_grouping_across_projections():
+    # One lora_group for the batch, then the three fused-slice decode
+    # projections (the same indices) as lora_bgmv calls with LORA_FLAG_GROUPED
+    # on that workspace: two launches each, no grouping.  Each against the
+    # oracle.
+    probs = W.config(3)
+    for p in probs[1:]:
+        assert np.array_equal(p.idx, probs[0].idx)
+    devs = [Dev(p) for p in probs]
+    meta = devs[0].meta
+    ops.group(devs[0].idx, probs[0].S, meta)
+    before = _lib.load().lora_launch_count()
+    for p, d in zip(probs, devs):
+        ops.bgmv(d.x, d.A, d.B, devs[0].idx, d.y, d.buf, meta, p.scale, y_col_off=p.col_off,
+                 grouped=True)
+    torch.cuda.synchronize()
+    assert _lib.load().lora_launch_count() - before == 2 * len(probs)
+    for p, d in zip(probs, devs):
+        buf_ref, cabs = oracle_shrink(p)
+        assert_buf_close(d.buf, buf_ref, cabs)
+        assert_y_close(p, d.y, oracle_expand(p, buf_ref), "y (end to end)")
+    assert ops.check_errors(meta) == _lib.LORA_OK
+
+
+def test_grouped_flag_with_a_stale_grouping_is_reported():
+    # The workspace grouped from another batch of the same size: the call
+    # reports it (LORA_ERR_BAD_INDEX) instead of using it silently.
+    p1 = W.config(3)[0]
+    p2 = W.make_problem(p1.name, p1.dtype, p1.T, p1.D, p1.r, p1.S, p1.d_out, p1.scale,
+                        seed=79, idx_kind="frac_neg", frac_neg=0.25)
+    assert not np.array_equal(p1.idx, p2.idx)
+    d1, d2 = Dev(p1), Dev(p2)
+    ops.group(d1.idx, p1.S, d1.meta)
+    ops.bgmv(d2.x, d2.A, d2.B, d2.idx, d2.y, d2.buf, d1.meta, p2.scale, y_col_off=p2.col_off,
+             grouped=True)
+    assert ops.check_errors(d1.meta) == _lib.LORA_ERR_BAD_INDEX
+
+
 def test_early_grouping_right_after_a_grouping_on_the_same_workspace():
     # A stand-alone grouping of one batch, then at once a three-launch
     # lora_bgmv call of another batch with LORA_FLAG_PDL_EARLY on the same
